@@ -1,0 +1,141 @@
+"""Oracle step drivers: replicated data parallelism (stage 0) and the ZeRO
+partitioned step (stages 1-3), on the CPU, with numpy.  Test infrastructure.
+
+Sources.  Mind-map page "ZeRO 真正在做什么：长期分开存，计算时临时拼齐":
+  - section "但 GPU 只存四分之一…": gradients are split again and sent to the
+    GPU responsible for each shard, which updates it and keeps it; before a
+    layer is computed the shards are exchanged so that every card briefly
+    holds the full layer, and the borrowed shards are dropped afterwards.
+  - "ZeRO 改的是训练状态的保存与通信方式，不是模型的学习算法": ZeRO changes
+    how state is stored and moved, not the learning algorithm.
+Concept page "ZeRO", section "为什么需要它": an update only needs all ranks to
+see one consistent full model logically; and table "三个阶段" (which states
+stay replicated at each stage: parameters at ZeRO-1/2, none at ZeRO-3, where
+parameters are all-gathered in execution order and released promptly).
+
+So the replicated step is the definition, and the partitioned step must reach
+exactly the same numbers: each owner runs the same elementwise core on its
+shard's columns, written through the partition maps of ``oracle.plan``.
+"""
+import numpy as np
+
+from . import core
+from .plan import Plan
+
+
+def step_replicated(nd, grads, w, m, v, adam, t, want_reduced=False):
+    """Stage 0: every rank keeps the full state and runs the full update.
+
+    grads: uint16 [nd, n] (rank r's bf16 gradient, logical order).
+    w, m, v: fp32 [nd, n], rank r's own full copy, updated in place.
+    Returns params uint16 [nd, n] (each rank's bf16 copy), reduced fp32 [n] of
+    rank 0 (or None), norm_sq, nonfinite (of rank 0's view).
+    """
+    n = grads.shape[1]
+    params = np.empty((nd, n), dtype=np.uint16)
+    red0 = None
+    norm0 = bad0 = None
+    for r in range(nd):
+        # all-reduce: every rank sums all ranks' gradients in rank order
+        p, red, norm, bad = core.update(grads, w[r], m[r], v[r], adam, t,
+                                        want_reduced=want_reduced)
+        params[r] = p
+        if r == 0:
+            red0, norm0, bad0 = red, norm, bad
+    return params, red0, norm0, bad0
+
+
+def step_partitioned(pl: Plan, grads, master, m, v, params, adam, t,
+                     reduced=None):
+    """Stages 1-3 over all Nd logical ranks.
+
+    grads: uint16 [nd, psi_pad], logical order (zero in the padding).
+    master, m, v, reduced: fp32 [nd * S], rank-major owner storage
+      (owner o's unit-u shard at o*S + O_u + [0, s_u)); updated in place.
+    params: uint16; stages 0-2: [nd, psi_pad] replicas, every rank's copy
+      rewritten with the owner's new values (the all-gather); stage 3:
+      [nd * S] owner shards only.
+    Returns (norm_sq, nonfinite) over all padded elements.
+    """
+    nd, S = pl.nd, pl.S
+    norm = 0.0
+    bad = 0
+    for o in range(nd):
+        for u in range(len(pl.unit_pad)):
+            s = pl.unit_shard[u]
+            lo = pl.unit_base[u] + o * s            # logical columns
+            st = o * S + pl.unit_offset[u]          # owner storage
+            cols = grads[:, lo:lo + s]
+            w_ = master[st:st + s]
+            m_ = m[st:st + s]
+            v_ = v[st:st + s]
+            p, red, nn, bb = core.update(cols, w_, m_, v_, adam, t,
+                                         want_reduced=reduced is not None)
+            norm += nn
+            bad += bb
+            if reduced is not None:
+                reduced[st:st + s] = red
+            if pl.stage == 3:
+                params[st:st + s] = p
+            else:
+                params[:, lo:lo + s] = p[None, :]
+    return norm, bad
+
+
+def step_owner_view(pl: Plan, owner, grads_owner, master, m, v, adam, t,
+                    want_reduced=False):
+    """One owner's part of the step.
+
+    grads_owner: uint16 [nd, S]: for every rank, its gradient on the columns
+      that `owner` owns, in the owner's storage order.
+    master, m, v: fp32 [S] (the owner's own state), updated in place.
+    Returns (params uint16 [S], reduced fp32 [S] or None, norm_sq, nonfinite).
+    """
+    p, red, nn, bb = core.update(grads_owner, master, m, v, adam, t,
+                                 want_reduced=want_reduced)
+    return p, red, nn, bb
+
+
+def owner_columns(pl: Plan, owner):
+    """Logical column indices that `owner` owns, in its storage order."""
+    parts = []
+    for u in range(len(pl.unit_pad)):
+        s = pl.unit_shard[u]
+        lo = pl.unit_base[u] + owner * s
+        parts.append(np.arange(lo, lo + s, dtype=np.int64))
+    return np.concatenate(parts)
+
+
+def gather_layer(pl: Plan, unit, owner_params):
+    """Stage 3 materialisation of one unit: concatenate the Nd owners' slices
+    of the unit in rank order and keep the first len_u (unpadded) elements.
+    owner_params: uint16 [nd * S] -> uint16 [len_u]."""
+    s = pl.unit_shard[unit]
+    pieces = []
+    for o in range(pl.nd):
+        st = o * pl.S + pl.unit_offset[unit]
+        pieces.append(owner_params[st:st + s])
+    return np.concatenate(pieces)[:pl.unit_len[unit]].copy()
+
+
+def logical_to_storage(pl: Plan, x_logical):
+    """[psi_pad] in logical order -> [nd * S] in rank-major owner storage."""
+    out = np.empty(pl.nd * pl.S, dtype=x_logical.dtype)
+    for o in range(pl.nd):
+        for u in range(len(pl.unit_pad)):
+            s = pl.unit_shard[u]
+            lo = pl.unit_base[u] + o * s
+            st = o * pl.S + pl.unit_offset[u]
+            out[st:st + s] = x_logical[lo:lo + s]
+    return out
+
+
+def storage_to_logical(pl: Plan, x_storage):
+    out = np.empty(pl.psi_pad, dtype=x_storage.dtype)
+    for o in range(pl.nd):
+        for u in range(len(pl.unit_pad)):
+            s = pl.unit_shard[u]
+            lo = pl.unit_base[u] + o * s
+            st = o * pl.S + pl.unit_offset[u]
+            out[lo:lo + s] = x_storage[st:st + s]
+    return out

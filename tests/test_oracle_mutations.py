@@ -1,0 +1,59 @@
+"""The pins catch plausible mistakes in the oracle's arithmetic.
+
+Each case plants one mistake in a copy of the C oracle (on the CPU, in a
+temporary directory), builds it, and runs the numeric pins of
+``test_oracle_pins.py`` against it: at least one pin must fail.
+"""
+import os
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "zero_oracle.c")
+
+MUTATIONS = {
+    "omb1_uses_beta2": ("sc[4] = (float)(1.0 - beta1);", "sc[4] = (float)(1.0 - beta2);"),
+    "eps_inside_sqrt": ("float root = sqrtf(v_new);", "float root = sqrtf(v_new + eps);"),
+    "no_bias_correction_1": ("sc[6] = (float)(lr / bc1);", "sc[6] = (float)lr;"),
+    "no_bias_correction_2": ("sc[7] = (float)(1.0 / sqrt(bc2));", "sc[7] = 1.0f;"),
+    "second_moment_missing_g": ("float v_new_part = v_g * g;", "float v_new_part = v_g;"),
+    "update_sign": ("float w_new = (*w) - delta;", "float w_new = (*w) + delta;"),
+    "grad_scale_dropped": ("float g = g_sum * grad_scale;", "float g = g_sum;"),
+    "sum_starts_at_zero": ("float s = bf16_bits_to_float(grads[e]);\n    for (uint32_t r = 1;",
+                           "float s = 0.0f;\n    for (uint32_t r = 0;"),
+    "sum_reverse_order": ("float x = bf16_bits_to_float(grads[(uint64_t)r * rank_stride + e]);",
+                          "float x = bf16_bits_to_float(grads[(uint64_t)(nd - r) * rank_stride + e]);"),
+    "bf16_truncates": ("uint32_t rounded = u + 0x7fffu + lsb;", "uint32_t rounded = u + 0u * lsb;"),
+    "bf16_ties_away": ("uint32_t rounded = u + 0x7fffu + lsb;", "uint32_t rounded = u + 0x8000u + 0u * lsb;"),
+    "beta1_for_v": ("float v_old = beta2 * (*v);", "float v_old = beta1 * (*v);"),
+}
+
+NUMERIC_PINS = ("reduce or bf16 or adam or closed_form or constant or zero_gradient "
+                "or norm or partitioned or owner_view")
+
+
+def _run_mutant(name, tmp):
+    old, new = MUTATIONS[name]
+    src = open(SRC, encoding="utf-8").read()
+    assert src.count(old) == 1, name
+    mutated = os.path.join(tmp, name + ".c")
+    with open(mutated, "w", encoding="utf-8") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(tmp, "lib" + name + ".so")
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+                    mutated, "-o", lib, "-lm"], check=True)
+    env = dict(os.environ, ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", NUMERIC_PINS],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    return r.returncode, r.stdout[-1500:]
+
+
+def test_planted_mistakes_are_caught(tmp_path):
+    names = sorted(MUTATIONS)
+    workers = max(1, min(len(names), (os.cpu_count() or 2) - 1))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        results = dict(zip(names, ex.map(lambda n: _run_mutant(n, str(tmp_path)), names)))
+    survived = {n: out for n, (rc, out) in results.items() if rc != 1}
+    assert not survived, survived
