@@ -1,0 +1,481 @@
+"""Benchmark of the ZeRO partitioned optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config c2] [--nd ND --bucket-mb MB]   # c5 points
+                    [--sweep OUT.jsonl]                      # whole c5 grid
+
+One step = the whole hot path over one batch of gradients: for every bucket,
+the fused reduce-scatter + owner Adam + all-gather kernel, then the
+gradient-norm / overflow reduction (stage 3 workloads add the forward and
+backward layer gathers).  The default workload is the GPT-2-small-shaped
+flat vector (124,439,808 parameters, Nd = 8 logical ranks, stage 2,
+25M-element buckets).  Inputs are resident in HBM when timing starts and one
+step touches ~7 GB, far more than the 126 MB L2, so no flush is needed.
+
+The metric is parameters updated per second (Gparams/s); the JSON line also
+carries the achieved HBM bandwidth of the dominant kernel against the measured
+B200 copy bandwidth, the CPU oracle timed on a bounded sample, an end-to-end
+number with host-resident gradients, and the SM clocks seen while timing.
+
+With N > 1 (torchrun), each rank runs the same single-GPU workload on its own
+GPU (the simulated ranks are HBM slices; there is no inter-GPU exchange), and
+the value is the sum over ranks of parameters over the slowest rank's time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Gparams/s per ZeRO step (RS+Adam+AG); achieved HBM GB/s vs B200 peak"
+UNIT = "Gparams/s"
+FALLBACK_HBM_GBS = 6650.0
+K1_PROFILE = os.path.join(ROOT, "profiles", "k_step_vec8_gpt2_small_nd8.md")
+K1_SOURCE = os.path.join(ROOT, "zero_partitioned_optimizer_step_b200", "csrc", "zero_step.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--nd", type=int, default=64)
+    ap.add_argument("--bucket-mb", type=int, default=64)
+    ap.add_argument("--sweep", default=None, help="write the c5 grid as JSON lines here")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--psi", type=int, default=None,
+                    help="override the parameter count (flat single-unit workloads only)")
+    return ap.parse_args()
+
+
+def get_cfg(args):
+    from zero_partitioned_optimizer_step_b200.configs import CONFIGS, c5_config
+    cfg = c5_config(args.nd, args.bucket_mb) if args.config == "c5" else dict(CONFIGS[args.config])
+    if args.psi is not None:
+        if cfg["units"] is not None or cfg["owner_view"] >= 0:
+            raise SystemExit("--psi applies to flat all-ranks workloads only")
+        cfg["psi"] = args.psi
+        cfg["workload"] = "flat vector psi=%d, Nd=%d, stage %d, %d-element buckets" % (
+            args.psi, cfg["nd"], cfg["stage"], cfg["bucket_elems"])
+    return cfg
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def k1_traffic_per_elem():
+    """dram bytes per element of the vector kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    try:
+        txt = open(K1_PROFILE, encoding="utf-8").read()
+        src_hash = hashlib.sha256(open(K1_SOURCE, "rb").read()).hexdigest()[:16]
+        m = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+        b = re.search(r"dram_bytes_per_element:\s*([0-9.eE+-]+)", txt)
+        if m and b and m.group(1) == src_hash:
+            return float(b.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed loop runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------- workload
+class Workload:
+    """Device buffers of one configuration, built from the seeded generators."""
+
+    def __init__(self, cfg, device):
+        import torch
+        import zero_partitioned_optimizer_step_b200 as Z
+        from zero_partitioned_optimizer_step_b200 import inputs
+        self.Z, self.torch = Z, torch
+        self.cfg = cfg
+        self.dev = device
+        nd, stage, owner = cfg["nd"], cfg["stage"], cfg["owner_view"]
+        self.lp = Z.zero_plan(cfg["psi"], nd, stage, cfg["bucket_elems"], unit_elems=cfg["units"])
+        self.units = self.lp.units()
+        self.S, self.psi_pad = self.lp.S, self.lp.psi_pad
+        self.adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
+        unit_len = [u[0] for u in self.units]
+        unit_pad = [u[1] for u in self.units]
+        if owner >= 0:
+            n = self.S
+            real = min(max(cfg["psi"] - owner * n, 0), n)
+            self.G = inputs.grads(nd, [real], [n], cfg["sigma"], cfg["id"], 1, device)
+            self.w = inputs.master_logical([real], [n], cfg["id"], device)
+        else:
+            n = nd * self.S
+            self.G = inputs.grads(nd, unit_len, unit_pad, cfg["sigma"], cfg["id"], 1, device,
+                                  outlier_frac=cfg["outlier_frac"])
+            w_log = inputs.master_logical(unit_len, unit_pad, cfg["id"], device)
+            self.w = torch.empty(n, dtype=torch.float32, device=device)
+            for o in range(nd):
+                for (ln, P, s, U, O) in self.units:
+                    self.w[o * self.S + O:o * self.S + O + s] = w_log[U + o * s:U + (o + 1) * s]
+            del w_log
+        self.m = torch.zeros(n, dtype=torch.float32, device=device)
+        self.v = torch.zeros(n, dtype=torch.float32, device=device)
+        self.replicas = owner < 0 and stage <= 2
+        if self.replicas:
+            self.params = torch.empty((nd, self.psi_pad), dtype=torch.bfloat16, device=device)
+        else:
+            self.params = torch.empty(n, dtype=torch.bfloat16, device=device)
+        self.norm = torch.zeros(1, dtype=torch.float64, device=device)
+        self.ovf = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = Z.workspace_for(self.lp, device)
+        self.layer = None
+        if stage == 3 and owner < 0:
+            self.layer = torch.empty(max(unit_len), dtype=torch.bfloat16, device=device)
+        self.owner = owner
+        flags = Z.ZERO_BYTES_FLAG_OWNER_VIEW if owner >= 0 else 0
+        self.step_bytes = Z.zero_bytes_moved(self.lp, Z.ZERO_BYTES_HBM_STEP, flags)
+        self.gather_bytes = (Z.zero_bytes_moved(self.lp, Z.ZERO_BYTES_HBM_GATHER_STEP)
+                             if self.layer is not None else 0)
+        self.elems = self.S if owner >= 0 else self.psi_pad
+        self.params_per_step = (min(max(cfg["psi"] - owner * self.S, 0), self.S)
+                                if owner >= 0 else cfg["psi"])
+        self.nb = self.lp.n_buckets
+
+    def bucket_elems(self, b):
+        """Elements bucket b processes (the owner's part in the owner view)."""
+        _, lo, hi = self.lp.query(self.Z.ZERO_Q_BUCKET_UNIT, b), \
+            self.lp.query(self.Z.ZERO_Q_BUCKET_BEGIN, b), self.lp.query(self.Z.ZERO_Q_BUCKET_END, b)
+        if self.owner < 0:
+            return hi - lo
+        u = self.lp.query(self.Z.ZERO_Q_BUCKET_UNIT, b)
+        ln, P, s, U, O = self.units[u]
+        a = U + self.owner * s
+        return max(0, min(hi, a + s) - max(lo, a))
+
+    def step(self, t, stream, events=None):
+        """One step; with `events` (list of nb+1 CUDA events) each bucket's
+        launch is bracketed so the vector kernel can be timed per launch."""
+        Z = self.Z
+        kw = dict(grad_norm_sq=self.norm, overflow=self.ovf, workspace=self.ws,
+                  owner_view=self.owner, stream=stream)
+        if events is None:
+            Z.zero_step(self.lp, self.G, self.w, self.m, self.v, self.params, self.adam, t, **kw)
+        else:
+            for b in range(self.nb):
+                events[b].record(stream)
+                Z.zero_step_buckets(self.lp, self.G, self.w, self.m, self.v, self.params,
+                                    self.adam, t, b, 1, **kw)
+            events[self.nb].record(stream)
+        if self.layer is not None:
+            n_units = len(self.units)
+            for u in list(range(n_units)) + list(reversed(range(n_units))):
+                Z.zero_gather_layer(self.lp, u, self.params, self.layer[:self.units[u][0]], stream)
+                Z.zero_release_layer(self.lp, u)
+
+    def launches_per_step(self):
+        n = sum(1 for b in range(self.nb) if self.bucket_elems(b) > 0)
+        n += 1  # norm / overflow finalize
+        if self.layer is not None:
+            n += 2 * len(self.units)
+        return n
+
+
+# ----------------------------------------------------------------- arms
+def cpu_baseline(wl, budget_s=12.0):
+    """The oracle, as it stands, on a bounded sample of the same workload:
+    consecutive 2^22-column windows of the step (all Nd gradient rows and the
+    state of those columns), until ~budget_s of single-threaded CPU time."""
+    import numpy as np
+    import torch
+    from oracle import core
+    win = min(1 << 22, wl.elems)
+    done, wins, t_compute = 0, 0, 0.0
+    while t_compute < budget_s and done < wl.elems:
+        lo = (wins * win) % max(1, wl.elems - win + 1)
+        G = wl.G[:, lo:lo + win].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+        w = wl.w[lo:lo + win].cpu().numpy()
+        m = wl.m[lo:lo + win].cpu().numpy()
+        v = wl.v[lo:lo + win].cpu().numpy()
+        t1 = time.perf_counter()
+        core.update(G, w, m, v, wl.adam, 1)
+        t_compute += time.perf_counter() - t1
+        done += win
+        wins += 1
+    return {"value": done / t_compute / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d windows of %d columns x %d gradient rows (%d params, %.1f s of "
+                      "single-threaded oracle time; host copies not timed)"
+                      % (wins, win, wl.cfg["nd"], done, t_compute)}
+
+
+def run_reference(args, cfg):
+    """Reference arm: the CPU oracle timed on the host cores, K steps of a
+    bounded sample (2^22 columns of the workload, all Nd gradient rows)."""
+    import numpy as np
+    import torch
+    from oracle import core
+    from zero_partitioned_optimizer_step_b200 import inputs
+    nd = cfg["nd"]
+    n = 1 << 22
+    G = inputs.grads(nd, [n], [n], cfg["sigma"], cfg["id"], 1, "cpu",
+                     outlier_frac=cfg["outlier_frac"])
+    G = G.view(torch.int16).numpy().view(np.uint16)
+    w = inputs.master_logical([n], [n], cfg["id"], "cpu").numpy()
+    m = np.zeros(n, np.float32)
+    v = np.zeros(n, np.float32)
+    adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
+    for t in range(1, args.warmup + 1):
+        core.update(G, w, m, v, adam, t)
+    t0 = time.perf_counter()
+    for t in range(args.warmup + 1, args.warmup + args.steps + 1):
+        core.update(G, w, m, v, adam, t)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt / 1e9
+    sample = ("%d columns x %d gradient rows of %s, per step" % (n, nd, cfg["workload"]))
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": cfg["workload"], "sample_columns": n},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_ours(args, cfg, rank, world, dist):
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = Workload(cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+    # warm-up (also builds the per-device launch grid)
+    for t in range(1, args.warmup + 1):
+        wl.step(t, stream)
+    torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(wl.nb + 1)]
+              for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index).start()
+    time.sleep(0.2)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    t0 = args.warmup + 1
+    for k in range(args.steps):
+        wl.step(t0 + k, stream, events[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed = start.elapsed_time(end) / 1e3
+    # dominant kernel: the fused bucket kernel, timed per launch
+    k1_time = 0.0
+    k1_elems = 0
+    for k in range(args.steps):
+        for b in range(wl.nb):
+            if wl.bucket_elems(b) == 0:
+                continue
+            k1_time += events[k][b].elapsed_time(events[k][b + 1]) / 1e3
+            k1_elems += wl.bucket_elems(b)
+    if dist is not None:
+        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # end to end through the public API: gradients from pinned host memory
+    # every step, the step, the norm and overflow flag read back every step
+    e2e = None
+    if not args.no_e2e:
+        e2e = _e2e(args, wl, stream, dev, world, dist, t0 + args.steps)
+    if rank != 0:
+        return None
+    return _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e)
+
+
+def _e2e(args, wl, stream, dev, world, dist, t_first):
+    import torch
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    Gh = wl.G.cpu().pin_memory()
+    out_h = torch.empty(2, dtype=torch.float64).pin_memory()
+    ovf_h = torch.empty(1, dtype=torch.int32).pin_memory()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for k in range(e2e_steps):
+        wl.G.copy_(Gh, non_blocking=True)
+        wl.step(t_first + k, stream)
+        out_h[:1].copy_(wl.norm, non_blocking=True)
+        ovf_h.copy_(wl.ovf, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_t = e0.elapsed_time(e1) / 1e3
+    if dist is not None:
+        t = torch.tensor([e2e_t], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_t = float(t.item())
+    return {"value": world * wl.params_per_step * e2e_steps / e2e_t / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": Gh.numel() * Gh.element_size(),
+            "d2h_bytes_per_step": 8 + 4, "steps": e2e_steps}
+
+
+def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
+    peak, peak_kind = measured_peak()
+    per_elem = wl.step_bytes / wl.elems
+    k1_bytes = per_elem * k1_elems
+    achieved = k1_bytes / k1_time / 1e9
+    n_launch = args.steps * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
+    tr = k1_traffic_per_elem() if (args.config == "c2" and args.psi is None) else None
+    roof = {"kernel": "k_step_vec8 (fused reduce-scatter + Adam + all-gather, one bucket)",
+            "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
+            "traffic": None if tr is None else tr * k1_elems / n_launch,
+            "algorithmic_bytes_per_launch": k1_bytes / n_launch,
+            "avg_launch_ms": k1_time / n_launch * 1e3}
+    step_bytes = wl.step_bytes + wl.gather_bytes
+    value = world * wl.params_per_step * args.steps / elapsed / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg["workload"], "psi": cfg["psi"], "nd": cfg["nd"],
+                   "stage": cfg["stage"], "bucket_elems": cfg["bucket_elems"],
+                   "owner_view": cfg["owner_view"], "buckets": wl.nb,
+                   "hbm_bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2 (%.2f GB touched per step, L2 126 MB); no flush"
+                         % (step_bytes / 1e9)},
+        "hbm_gbs": step_bytes / (elapsed / args.steps) / 1e9,
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": wl.launches_per_step() * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        out["cpu_baseline"] = cpu_baseline(wl)
+    return out
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    cfg = get_cfg(args)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.sweep:
+            from zero_partitioned_optimizer_step_b200.configs import c5_config
+            with open(args.sweep, "w") as f:
+                for nd in (2, 4, 8, 16, 64):
+                    for mb in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512):
+                        a = argparse.Namespace(**vars(args))
+                        a.config = "c5"
+                        a.no_cpu_baseline = True
+                        a.no_e2e = True
+                        res = run_ours(a, c5_config(nd, mb), rank, world, dist)
+                        if res is not None:
+                            res["config"]["bucket_mb"] = mb
+                            f.write(json.dumps(res) + "\n")
+                            f.flush()
+                            print(json.dumps({"nd": nd, "mb": mb, "value": res["value"],
+                                              "hbm_gbs": res["roofline"]["achieved"]}), flush=True)
+                        import torch
+                        torch.cuda.empty_cache()
+            return 0
+        res = run_ours(args, cfg, rank, world, dist)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

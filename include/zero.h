@@ -1,0 +1,271 @@
+/*
+ * zero.h -- C ABI of libzero.so, the B200 (sm_100a) ZeRO partitioned
+ * mixed-precision Adam step.
+ *
+ * What the library computes.  Nd data-parallel ranks are simulated as slices
+ * of one GPU's memory.  One step, per bucket of the flat parameter vector:
+ *   1. reduce-scatter (ZeRO "Pg"): for every padded element, the fp32 sum of
+ *      the Nd ranks' bf16 gradients, added in rank order 0, 1, ..., Nd-1
+ *      starting from rank 0's value; only the owner of the element keeps it;
+ *   2. owner Adam (ZeRO "Pos"): the owner updates its fp32 master weight and
+ *      its fp32 first and second moments (K = 12 bytes of state per element);
+ *   3. all-gather: the new bf16 parameter is written to every rank's full
+ *      replica (stages 0-2), or to the owner's shard only (stage 3), from
+ *      where zero_gather_layer() materialises one layer at a time.
+ * All of it runs in hand-written CUDA kernels; there is no CPU path.
+ *
+ * Sources (three web pages about ZeRO, arXiv 1910.02054):
+ *  [MM] mind-map page "ZeRO 真正在做什么：长期分开存，计算时临时拼齐"
+ *       (paperbridge.wiki): the four-GPU A/B/C/D example; the loop "store
+ *       apart -> gather the current layer -> compute -> split again"; the
+ *       stage list; the 7.5B / Nd=64 memory estimate; the 2 Psi / 3 Psi
+ *       communication volumes; the glossary (all-gather, reduce-scatter,
+ *       temporary materialisation).
+ *  [CP] concept page "ZeRO" (papers.lqhl.me): "为什么需要它" (mixed-precision
+ *       Adam state), table "三个阶段" (what each stage shards), "关键设计取舍"
+ *       item 1 (bucket size versus launch latency), the remark that ZeRO-3
+ *       still materialises layers and that unreleased layers make peaks.
+ *  [GG] gptget.net summary page of arXiv 1910.02054: stages Pos, Pg, Pp.
+ *
+ * Layouts (element counts; A = align_elems; u = unit, r = rank):
+ *   P_u = ceil(len_u / (Nd*A)) * Nd*A    padded unit length
+ *   s_u = P_u / Nd                       elements of unit u each rank owns
+ *   U_u = sum_{u'<u} P_u'                unit u's start in the logical vector
+ *   O_u = sum_{u'<u} s_u'                unit u's start inside a rank's block
+ *   psi_pad = sum P_u,  S = sum s_u      (one unit: S = psi_pad / Nd)
+ *   logical order:  unit after unit, each padded with zeros.
+ *   owner storage:  rank-major [Nd][S]; rank o's slice of unit u (logical
+ *                   U_u + o*s_u + i, 0 <= i < s_u) sits at o*S + O_u + i.
+ *   With one unit the two orders coincide.
+ *
+ * Ownership.  The caller allocates, owns and frees every device buffer and
+ * the stream; the library keeps only the host-side plan (maps, bucket table,
+ * live-layer bookkeeping).  Device scratch, when needed, is the caller's
+ * `workspace` (size: zero_plan_query(ZERO_Q_WORKSPACE_BYTES)).
+ *
+ * Errors.  No call aborts or prints.  Every call returns a status; the text of
+ * the last failure on the calling thread is zero_last_error().  Invalid
+ * arguments (NULL or non-16-byte-aligned device pointers, bad descriptor,
+ * t = 0, index out of range) give ZERO_EINVAL before anything is launched.
+ * Liveness violations give ZERO_ESTATE.  A failed launch gives ZERO_ECUDA;
+ * faults inside a kernel are asynchronous and surface on a later CUDA call.
+ *
+ * Streams.  `stream` is a cudaStream_t passed as void*; NULL is the legacy
+ * default stream.  Launches are asynchronous; nothing synchronises.
+ * Threads.  A plan may be shared by threads for zero_step*() and queries;
+ * zero_gather_layer()/zero_release_layer() serialise on the plan internally.
+ */
+#ifndef ZERO_H_
+#define ZERO_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZERO_ABI_VERSION 1
+
+typedef enum zero_status {
+    ZERO_OK = 0,
+    ZERO_EINVAL = 1,   /* invalid argument */
+    ZERO_ENOMEM = 2,   /* host allocation failed */
+    ZERO_ECUDA = 3,    /* CUDA runtime or launch error */
+    ZERO_ESTATE = 4,   /* not allowed in the current live-layer state */
+    ZERO_ETIMEOUT = 5  /* a bounded device wait gave up */
+} zero_status_t;
+
+typedef struct zero_plan zero_plan_t;      /* opaque, host memory */
+
+/* Partition descriptor.  Zero-valued optional fields take their default. */
+typedef struct zero_plan_desc {
+    uint64_t psi;          /* parameters; = sum(unit_elems) when units given */
+    uint32_t nd;           /* logical data-parallel ranks, >= 1 */
+    uint32_t stage;        /* 0 replicated DP, 1 Pos, 2 Pos+g, 3 Pos+g+p */
+    uint64_t bucket_elems; /* padded elements per bucket, >= 1 */
+    uint32_t align_elems;  /* A; each unit padded to a multiple of Nd*A; 0 -> 64 */
+    uint32_t k_bytes;      /* optimizer bytes/param of the memory model; 0 -> 12 */
+    uint32_t n_units;      /* 0 -> one unit of psi elements */
+    uint32_t max_live;     /* stage 3: units gathered at once; 0 -> 1 */
+    const uint64_t *unit_elems; /* n_units lengths (host; copied), or NULL */
+} zero_plan_desc_t;
+
+/* Build a plan: shard sizes, offsets, padding, bucket table, accounting.
+ * Source: [MM] four-GPU example (GPU i keeps block i) and section "但 GPU
+ * 只存四分之一…" (each card keeps a shard of the current layer); [CP] table
+ * "三个阶段"; [CP] "关键设计取舍" item 1 (buckets).  Units are cut into Nd
+ * equal contiguous shards in rank order, after zero padding to a multiple of
+ * Nd*A; a bucket is a contiguous range of bucket_elems padded elements of the
+ * logical vector, cut at unit boundaries (a unit's last bucket is short).
+ * Host only.  *out receives a new plan owned by the caller (free with
+ * zero_plan_destroy).  ZERO_EINVAL: NULL argument, psi/nd/bucket_elems = 0,
+ * stage > 3, unit lengths that are zero or do not sum to psi, or sizes that
+ * overflow 64 bits.  ZERO_ENOMEM: host allocation failed. */
+zero_status_t zero_plan(const zero_plan_desc_t *desc, zero_plan_t **out);
+
+/* Free a plan (NULL is ignored).  Device buffers are the caller's. */
+void zero_plan_destroy(zero_plan_t *plan);
+
+typedef enum zero_query {
+    ZERO_Q_PSI = 0,          /* psi */
+    ZERO_Q_PSI_PAD = 1,      /* psi_pad */
+    ZERO_Q_S = 2,            /* S, elements one rank owns */
+    ZERO_Q_ND = 3,
+    ZERO_Q_STAGE = 4,
+    ZERO_Q_N_UNITS = 5,
+    ZERO_Q_UNIT_LEN = 6,     /* idx = u: len_u */
+    ZERO_Q_UNIT_PAD = 7,     /* idx = u: P_u */
+    ZERO_Q_UNIT_SHARD = 8,   /* idx = u: s_u */
+    ZERO_Q_UNIT_BASE = 9,    /* idx = u: U_u */
+    ZERO_Q_UNIT_OFFSET = 10, /* idx = u: O_u */
+    ZERO_Q_N_BUCKETS = 11,
+    ZERO_Q_BUCKET_UNIT = 12, /* idx = b: unit of bucket b */
+    ZERO_Q_BUCKET_BEGIN = 13,/* idx = b: logical begin (inclusive) */
+    ZERO_Q_BUCKET_END = 14,  /* idx = b: logical end (exclusive) */
+    ZERO_Q_OWNER = 15,       /* idx = logical p: owner rank */
+    ZERO_Q_OWNER_OFFSET = 16,/* idx = logical p: offset in the owner's S block */
+    ZERO_Q_MEM_BYTES_PER_RANK = 17, /* idx = stage 0..3: resident model-state
+                                bytes per rank with padded sizes:
+                                (4+K)psi_pad, 4psi_pad+K S, 2psi_pad+(2+K)S,
+                                (4+K)S.  With A = 1 and Nd | psi these are the
+                                [MM] closed forms exactly. */
+    ZERO_Q_WORKSPACE_BYTES = 18,/* device workspace zero_step needs when it
+                                   reports the gradient norm or overflow */
+    ZERO_Q_LIVE_UNITS = 19,     /* stage 3: units gathered and not released */
+    ZERO_Q_PEAK_LIVE_UNITS = 20,
+    ZERO_Q_PEAK_LIVE_BYTES = 21,/* bf16 bytes of the largest live set seen */
+    ZERO_Q_IS_LIVE = 22,        /* idx = u: 1 if unit u is live */
+    ZERO_Q_MAX_LIVE = 23,
+    ZERO_Q_ALIGN = 24,
+    ZERO_Q_BUCKET_ELEMS = 25
+} zero_query_t;
+
+/* Read one value of the plan into *out.  Host only.  ZERO_EINVAL: NULL
+ * argument, unknown `what`, or `idx` out of range. */
+zero_status_t zero_plan_query(const zero_plan_t *plan, zero_query_t what,
+                              uint64_t idx, uint64_t *out);
+
+/* Adam hyperparameters (double, as optimizer settings usually are).  Per
+ * element, with constants rounded once to fp32 (b1, b2, eps, grad_scale,
+ * 1-b1, 1-b2, step = lr/(1-b1^t), ibc2 = 1/sqrt(1-b2^t), powers by pow()):
+ *   g = g_sum*grad_scale;  m = b1*m + (1-b1)*g;  v = b2*v + ((1-b2)*g)*g;
+ *   w = w - step * (m / (sqrt(v)*ibc2 + eps));  p = bf16_rne(w)
+ * each operation a separate round-to-nearest fp32 operation (no FMA).
+ * This is textbook Adam (bias-corrected, eps outside the root, no weight
+ * decay); [CP] "为什么需要它" names the state, the pages give no formula. */
+typedef struct zero_adam {
+    double lr, beta1, beta2, eps;
+    double grad_scale;     /* 1/Nd averages the summed gradient */
+} zero_adam_t;
+
+/* Device buffers of one step (all device pointers, 16-byte aligned). */
+typedef struct zero_bufs {
+    const void *grads;     /* bf16 [Nd][grad_stride]; all-ranks view: rank r's
+                              full gradient in logical order (padding zero);
+                              owner view: rank r's gradient on the owner's
+                              columns, in the owner's storage order */
+    uint64_t grad_stride;  /* elements between ranks: >= psi_pad (all ranks)
+                              or >= S (owner view) */
+    float *master;         /* fp32 master weights: [Nd*S] owner storage
+                              (all ranks) or [S] (owner view); in/out */
+    float *exp_avg;        /* fp32 m, same layout; in/out */
+    float *exp_avg_sq;     /* fp32 v, same layout; in/out */
+    void *params;          /* bf16 out.  Stages 0-2, all ranks: Nd replica
+                              rows [Nd][param_stride] in logical order; stage 3
+                              or owner view: owner shards in storage order */
+    uint64_t param_stride; /* replica rows only: >= psi_pad */
+    float *reduced_grad;   /* optional fp32 out, layout of master: the
+                              reduce-scatter result g_sum (before grad_scale) */
+    double *grad_norm_sq;  /* optional device scalar out: sum of g_sum^2 over
+                              the elements processed by the call */
+    int32_t *overflow;     /* optional device scalar out: 1 if any g_sum is
+                              inf or NaN, else 0 */
+    void *workspace;       /* device scratch, needed iff grad_norm_sq or
+                              overflow is set; caller-owned */
+    uint64_t workspace_bytes;
+    int32_t owner_view;    /* -1: all Nd ranks; o in [0,Nd): rank o only */
+} zero_bufs_t;
+
+/* One full step: every bucket in order, then (if asked) the norm/overflow.
+ * Source: [MM] section "但 GPU 只存四分之一…" (gradients are split back to
+ * the GPU responsible for the shard, which updates and keeps it; shards are
+ * exchanged so each card briefly holds the full layer); [CP] table
+ * "三个阶段" rows ZeRO-1/2/3; [MM] "ZeRO 改的是…不是模型的学习算法" (the
+ * result equals replicated data-parallel Adam).  t is the 1-based step.
+ * The padding of `grads` must be zero; the padding of the state then stays 0.
+ * ZERO_EINVAL: NULL/misaligned pointer, short stride, t = 0, owner_view out
+ * of range, norm or overflow without a big enough workspace, non-finite lr,
+ * beta outside [0,1).  ZERO_ECUDA: launch failure. */
+zero_status_t zero_step(const zero_plan_t *plan, const zero_bufs_t *bufs,
+                        const zero_adam_t *adam, uint64_t t, void *stream);
+
+/* Buckets [first_bucket, first_bucket + n_buckets) of a step, for callers
+ * that launch each bucket as soon as its gradients exist ([CP] "关键设计取舍"
+ * item 1).  The norm/overflow workspace is reset by the call that contains
+ * bucket 0 and reported by the call that contains the last bucket; calls of
+ * one step must run in bucket order on one stream.  In the owner view,
+ * buckets the owner has no part of launch nothing.  Errors as zero_step,
+ * plus ZERO_EINVAL for a bucket range outside the plan. */
+zero_status_t zero_step_buckets(const zero_plan_t *plan,
+                                 const zero_bufs_t *bufs,
+                                 const zero_adam_t *adam, uint64_t t,
+                                 uint64_t first_bucket, uint64_t n_buckets,
+                                 void *stream);
+
+/* Stage 3: materialise unit `unit` -- copy the Nd owners' bf16 slices of it,
+ * in rank order, into full_layer[0 .. len_u) (padding dropped) -- and mark
+ * it live.  Source: [MM] glossary "临时物化" and "all-gather" (shards are
+ * briefly put together into the full parameters of the current layer);
+ * [CP] table "三个阶段" row ZeRO-3 (all-gather in execution order, release
+ * promptly).  owner_params: bf16 [Nd*S] owner storage (zero_step's params at
+ * stage 3); full_layer: bf16 [len_u], caller-owned.  ZERO_EINVAL: stage != 3,
+ * unit out of range, NULL/misaligned pointer.  ZERO_ESTATE: the unit is
+ * already live, or max_live units are live.  ZERO_ECUDA: launch failure (the
+ * unit is then not marked live). */
+zero_status_t zero_gather_layer(zero_plan_t *plan, uint32_t unit,
+                                const void *owner_params, void *full_layer,
+                                void *stream);
+
+/* Stage 3: release a live unit (its full_layer buffer may be reused once the
+ * work queued on it is done).  Source: [MM] glossary "临时物化" (no extra copy
+ * is kept after the computation); [CP] remark under "三个阶段" (unreleased
+ * layers form memory peaks).  Host only.  ZERO_EINVAL: unit out of range.
+ * ZERO_ESTATE: the unit is not live. */
+zero_status_t zero_release_layer(zero_plan_t *plan, uint32_t unit);
+
+typedef enum zero_bytes_kind {
+    ZERO_BYTES_COMM_ELEMS_PER_RANK = 0, /* ring model, elements one rank sends
+                                           per step: 2(Nd-1)S at stages 0-2,
+                                           3(Nd-1)S at stage 3 */
+    ZERO_BYTES_COMM_PER_RANK = 1,       /* the same in bytes (bf16) */
+    ZERO_BYTES_HBM_STEP = 2,            /* bytes zero_step moves in HBM */
+    ZERO_BYTES_HBM_GATHER_STEP = 3      /* bytes of the stage-3 gathers of one
+                                           step (2 per unit: 4 B/element) */
+} zero_bytes_kind_t;
+
+#define ZERO_BYTES_FLAG_OWNER_VIEW 1u    /* HBM_STEP of one owner's shard */
+#define ZERO_BYTES_FLAG_REDUCED 2u       /* HBM_STEP incl. reduced_grad writes */
+
+/* Accounting.  Source: [MM] "论文证据" (plain DP and gradient partitioning
+ * move 2 Psi per step, parameter partitioning 3 Psi, about 1.5 times).
+ * HBM_STEP = n*(2Nd + 24 + w) [+4n], n = psi_pad (S in the owner view),
+ * w = 2Nd for replicas (stages 0-2, all ranks) else 2.  ZERO_EINVAL: NULL
+ * argument or unknown kind. */
+zero_status_t zero_bytes_moved(const zero_plan_t *plan, zero_bytes_kind_t kind,
+                               uint32_t flags, uint64_t *out);
+
+/* Static text of a status code. */
+const char *zero_status_str(zero_status_t status);
+
+/* Text of the last failure on the calling thread ("" if none).  Valid until
+ * the next call on that thread. */
+const char *zero_last_error(void);
+
+/* ZERO_ABI_VERSION of the loaded library. */
+uint32_t zero_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_H_ */

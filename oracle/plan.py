@@ -183,3 +183,17 @@ def hbm_gather_bytes(pl: Plan, gathers_per_unit: int = 2) -> int:
     """Stage 3 materialisation: read 2 B and write 2 B per element of each
     unit, `gathers_per_unit` times per step (forward, then backward)."""
     return gathers_per_unit * sum(4 * n for n in pl.unit_len)
+
+
+def storage_index(pl: Plan, cols):
+    """Vector form of `locate`: logical indices -> rank-major storage index
+    (owner * S + offset in the owner's block).  numpy int64 in and out."""
+    import numpy as np
+    cols = np.asarray(cols, dtype=np.int64)
+    base = np.asarray(pl.unit_base, dtype=np.int64)
+    u = np.searchsorted(base, cols, side="right") - 1
+    j = cols - base[u]
+    s = np.asarray(pl.unit_shard, dtype=np.int64)[u]
+    owner = j // s
+    off = np.asarray(pl.unit_offset, dtype=np.int64)[u] + (j - owner * s)
+    return owner * pl.S + off

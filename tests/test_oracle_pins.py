@@ -154,6 +154,9 @@ def test_maps_brute_force_small():
                 for u, n in enumerate(units):
                     assert 0 <= pl.unit_pad[u] - n < nd * align
                 assert pl.buckets == buckets
+                sidx = P.storage_index(pl, range(len(logical)))
+                assert [int(x) for x in sidx] == [where[p][0] * S + where[p][1]
+                                                  for p in range(len(logical))]
                 cases += 1
     assert cases > 1000
 

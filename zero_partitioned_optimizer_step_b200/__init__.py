@@ -1,1 +1,304 @@
-"""B200-native ZeRO partitioned optimizer step (package placeholder)."""
+"""B200-native ZeRO partitioned mixed-precision Adam step.
+
+Thin Python binding of ``libzero.so`` (C ABI in ``include/zero.h``): the same
+entry points, with torch tensors turned into device pointers and the current
+torch stream passed as the CUDA stream.  Every step of the computation runs
+in the library's sm_100a kernels; there is no Python or CPU fallback -- if the
+library is missing, every call raises.
+
+    plan = zero_plan(psi, nd, stage, bucket_elems, unit_elems=[...])
+    zero_step(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t)
+    zero_gather_layer(plan, u, owner_params, full_layer)   # stage 3
+    zero_release_layer(plan, u)
+"""
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libzero.so")
+
+# status codes (zero_status_t)
+ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ETIMEOUT = range(6)
+
+# queries (zero_query_t)
+(ZERO_Q_PSI, ZERO_Q_PSI_PAD, ZERO_Q_S, ZERO_Q_ND, ZERO_Q_STAGE, ZERO_Q_N_UNITS,
+ ZERO_Q_UNIT_LEN, ZERO_Q_UNIT_PAD, ZERO_Q_UNIT_SHARD, ZERO_Q_UNIT_BASE,
+ ZERO_Q_UNIT_OFFSET, ZERO_Q_N_BUCKETS, ZERO_Q_BUCKET_UNIT, ZERO_Q_BUCKET_BEGIN,
+ ZERO_Q_BUCKET_END, ZERO_Q_OWNER, ZERO_Q_OWNER_OFFSET, ZERO_Q_MEM_BYTES_PER_RANK,
+ ZERO_Q_WORKSPACE_BYTES, ZERO_Q_LIVE_UNITS, ZERO_Q_PEAK_LIVE_UNITS,
+ ZERO_Q_PEAK_LIVE_BYTES, ZERO_Q_IS_LIVE, ZERO_Q_MAX_LIVE, ZERO_Q_ALIGN,
+ ZERO_Q_BUCKET_ELEMS) = range(26)
+
+# accounting kinds (zero_bytes_kind_t) and flags
+(ZERO_BYTES_COMM_ELEMS_PER_RANK, ZERO_BYTES_COMM_PER_RANK, ZERO_BYTES_HBM_STEP,
+ ZERO_BYTES_HBM_GATHER_STEP) = range(4)
+ZERO_BYTES_FLAG_OWNER_VIEW = 1
+ZERO_BYTES_FLAG_REDUCED = 2
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("%s (%s)" % (message, status))
+        self.status = status
+
+
+class _PlanDesc(ctypes.Structure):
+    _fields_ = [("psi", ctypes.c_uint64), ("nd", ctypes.c_uint32),
+                ("stage", ctypes.c_uint32), ("bucket_elems", ctypes.c_uint64),
+                ("align_elems", ctypes.c_uint32), ("k_bytes", ctypes.c_uint32),
+                ("n_units", ctypes.c_uint32), ("max_live", ctypes.c_uint32),
+                ("unit_elems", ctypes.POINTER(ctypes.c_uint64))]
+
+
+class _Adam(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
+                ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
+                ("grad_scale", ctypes.c_double)]
+
+
+class _Bufs(ctypes.Structure):
+    _fields_ = [("grads", ctypes.c_void_p), ("grad_stride", ctypes.c_uint64),
+                ("master", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p),
+                ("exp_avg_sq", ctypes.c_void_p), ("params", ctypes.c_void_p),
+                ("param_stride", ctypes.c_uint64), ("reduced_grad", ctypes.c_void_p),
+                ("grad_norm_sq", ctypes.c_void_p), ("overflow", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
+                ("owner_view", ctypes.c_int32)]
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded libzero.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libzero.so is missing (%s); build it with "
+                "`python -m zero_partitioned_optimizer_step_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        st = ctypes.c_int
+        vp = ctypes.c_void_p
+        u64 = ctypes.c_uint64
+        L.zero_plan.restype = st
+        L.zero_plan.argtypes = [ctypes.POINTER(_PlanDesc), ctypes.POINTER(vp)]
+        L.zero_plan_destroy.restype = None
+        L.zero_plan_destroy.argtypes = [vp]
+        L.zero_plan_query.restype = st
+        L.zero_plan_query.argtypes = [vp, ctypes.c_int, u64, ctypes.POINTER(u64)]
+        L.zero_step.restype = st
+        L.zero_step.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam), u64, vp]
+        L.zero_step_buckets.restype = st
+        L.zero_step_buckets.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam),
+                                        u64, u64, u64, vp]
+        L.zero_gather_layer.restype = st
+        L.zero_gather_layer.argtypes = [vp, ctypes.c_uint32, vp, vp, vp]
+        L.zero_release_layer.restype = st
+        L.zero_release_layer.argtypes = [vp, ctypes.c_uint32]
+        L.zero_bytes_moved.restype = st
+        L.zero_bytes_moved.argtypes = [vp, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(u64)]
+        L.zero_status_str.restype = ctypes.c_char_p
+        L.zero_status_str.argtypes = [ctypes.c_int]
+        L.zero_last_error.restype = ctypes.c_char_p
+        L.zero_last_error.argtypes = []
+        L.zero_abi_version.restype = ctypes.c_uint32
+        L.zero_abi_version.argtypes = []
+        _LIB = L
+    return _LIB
+
+
+def _check(status):
+    if status != ZERO_OK:
+        L = lib()
+        msg = L.zero_last_error().decode() or L.zero_status_str(status).decode()
+        raise ZeroError(status, msg)
+
+
+class Plan:
+    """Owns a zero_plan_t handle."""
+
+    def __init__(self, handle):
+        self._h = ctypes.c_void_p(handle)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def query(self, what, idx=0):
+        return zero_plan_query(self, what, idx)
+
+    # convenience views of the plan
+    @property
+    def psi(self):
+        return self.query(ZERO_Q_PSI)
+
+    @property
+    def psi_pad(self):
+        return self.query(ZERO_Q_PSI_PAD)
+
+    @property
+    def S(self):
+        return self.query(ZERO_Q_S)
+
+    @property
+    def nd(self):
+        return self.query(ZERO_Q_ND)
+
+    @property
+    def stage(self):
+        return self.query(ZERO_Q_STAGE)
+
+    @property
+    def n_units(self):
+        return self.query(ZERO_Q_N_UNITS)
+
+    @property
+    def n_buckets(self):
+        return self.query(ZERO_Q_N_BUCKETS)
+
+    def units(self):
+        """[(len, pad, shard, base, offset)] per unit."""
+        return [tuple(self.query(q, u) for q in (ZERO_Q_UNIT_LEN, ZERO_Q_UNIT_PAD,
+                                                  ZERO_Q_UNIT_SHARD, ZERO_Q_UNIT_BASE,
+                                                  ZERO_Q_UNIT_OFFSET))
+                for u in range(self.n_units)]
+
+    def buckets(self):
+        """[(unit, begin, end)] per bucket (logical, end exclusive)."""
+        return [tuple(self.query(q, b) for q in (ZERO_Q_BUCKET_UNIT, ZERO_Q_BUCKET_BEGIN,
+                                                  ZERO_Q_BUCKET_END))
+                for b in range(self.n_buckets)]
+
+    def __del__(self):
+        h, self._h = getattr(self, "_h", None), None
+        if h and _LIB is not None:
+            _LIB.zero_plan_destroy(h)
+
+
+def zero_plan(psi, nd, stage, bucket_elems, align_elems=64, k_bytes=12,
+              unit_elems=None, max_live=1):
+    """Build a plan (see zero_plan in include/zero.h)."""
+    desc = _PlanDesc()
+    desc.psi = int(psi)
+    desc.nd = int(nd)
+    desc.stage = int(stage)
+    desc.bucket_elems = int(bucket_elems)
+    desc.align_elems = int(align_elems)
+    desc.k_bytes = int(k_bytes)
+    desc.max_live = int(max_live)
+    arr = None
+    if unit_elems:
+        arr = (ctypes.c_uint64 * len(unit_elems))(*[int(x) for x in unit_elems])
+        desc.n_units = len(unit_elems)
+        desc.unit_elems = arr
+    h = ctypes.c_void_p()
+    _check(lib().zero_plan(ctypes.byref(desc), ctypes.byref(h)))
+    return Plan(h.value)
+
+
+def zero_plan_query(plan, what, idx=0):
+    out = ctypes.c_uint64()
+    _check(lib().zero_plan_query(plan.handle, int(what), int(idx), ctypes.byref(out)))
+    return out.value
+
+
+def zero_bytes_moved(plan, kind, flags=0):
+    out = ctypes.c_uint64()
+    _check(lib().zero_bytes_moved(plan.handle, int(kind), int(flags), ctypes.byref(out)))
+    return out.value
+
+
+def zero_release_layer(plan, unit):
+    _check(lib().zero_release_layer(plan.handle, int(unit)))
+
+
+# ------------------------------------------------------------ device calls
+def _ptr(t, dtype=None, name="tensor"):
+    """Device pointer of a CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _row_stride(t, default):
+    if t is not None and t.dim() == 2:
+        if t.stride(1) != 1:
+            raise ValueError("rows must be contiguous")
+        return t.stride(0)
+    return default
+
+
+def make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, reduced_grad=None,
+              grad_norm_sq=None, overflow=None, workspace=None, owner_view=-1,
+              grad_stride=None, param_stride=None):
+    import torch
+    b = _Bufs()
+    b.grads = _ptr(grads, torch.bfloat16, "grads")
+    default_g = plan.S if owner_view >= 0 else plan.psi_pad
+    b.grad_stride = int(grad_stride if grad_stride is not None else _row_stride(grads, default_g))
+    b.master = _ptr(master, torch.float32, "master")
+    b.exp_avg = _ptr(exp_avg, torch.float32, "exp_avg")
+    b.exp_avg_sq = _ptr(exp_avg_sq, torch.float32, "exp_avg_sq")
+    b.params = _ptr(params, torch.bfloat16, "params")
+    b.param_stride = int(param_stride if param_stride is not None
+                         else _row_stride(params, plan.psi_pad))
+    b.reduced_grad = _ptr(reduced_grad, torch.float32, "reduced_grad")
+    b.grad_norm_sq = _ptr(grad_norm_sq, torch.float64, "grad_norm_sq")
+    b.overflow = _ptr(overflow, torch.int32, "overflow")
+    b.workspace = _ptr(workspace, None, "workspace")
+    b.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    b.owner_view = int(owner_view)
+    return b
+
+
+def make_adam(adam):
+    a = _Adam()
+    a.lr = float(adam["lr"])
+    a.beta1 = float(adam["beta1"])
+    a.beta2 = float(adam["beta2"])
+    a.eps = float(adam["eps"])
+    a.grad_scale = float(adam["grad_scale"])
+    return a
+
+
+def zero_step(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t, stream=None, **kw):
+    """One full step (all buckets, then the optional norm/overflow)."""
+    b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
+    _check(lib().zero_step(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
+                           int(t), _stream(stream)))
+
+
+def zero_step_buckets(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t,
+                      first_bucket, n_buckets, stream=None, **kw):
+    """Buckets [first_bucket, first_bucket + n_buckets) of step t."""
+    b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
+    _check(lib().zero_step_buckets(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
+                                   int(t), int(first_bucket), int(n_buckets), _stream(stream)))
+
+
+def zero_gather_layer(plan, unit, owner_params, full_layer, stream=None):
+    import torch
+    _check(lib().zero_gather_layer(plan.handle, int(unit),
+                                   _ptr(owner_params, torch.bfloat16, "owner_params"),
+                                   _ptr(full_layer, torch.bfloat16, "full_layer"),
+                                   _stream(stream)))
+
+
+def workspace_for(plan, device="cuda"):
+    """A caller-owned device workspace of the size the norm/overflow needs."""
+    import torch
+    return torch.empty(plan.query(ZERO_Q_WORKSPACE_BYTES), dtype=torch.uint8, device=device)
