@@ -250,17 +250,19 @@ class Workload:
 
 
 # ----------------------------------------------------------------- arms
-def cpu_baseline(wl, budget_s=12.0):
+def cpu_baseline(wl, budget_s=10.0):
     """The oracle, as it stands, on a bounded sample of the same workload:
     consecutive 2^22-column windows of the step (all Nd gradient rows and the
-    state of those columns), until ~budget_s of single-threaded CPU time."""
+    state of those columns, wrapping around), until ~budget_s of
+    single-threaded CPU time."""
     import numpy as np
     import torch
     from oracle import core
     win = min(1 << 22, wl.elems)
     done, wins, t_compute = 0, 0, 0.0
-    while t_compute < budget_s and done < wl.elems:
-        lo = (wins * win) % max(1, wl.elems - win + 1)
+    n_win = max(1, wl.elems // win)
+    while t_compute < budget_s:
+        lo = (wins % n_win) * win
         G = wl.G[:, lo:lo + win].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
         w = wl.w[lo:lo + win].cpu().numpy()
         m = wl.m[lo:lo + win].cpu().numpy()
