@@ -212,6 +212,26 @@ zero_status_t zero_step_buckets(const zero_plan_t *plan,
                                  uint64_t first_bucket, uint64_t n_buckets,
                                  void *stream);
 
+/* zero_step() without a caller-provided workspace, for callers that cannot
+ * allocate device memory (a runtime whose device memory is all handed out by
+ * its own pool up front, a plain C caller with no allocator of its own, code
+ * that must not allocate while it runs).  The paper has no counterpart: this
+ * is a packaging choice of this library.  The norm/overflow scratch lives in a
+ * 49,152-byte static array in device memory owned by the library, present on
+ * every GPU that loads it until the process exits; bufs->workspace and
+ * bufs->workspace_bytes are ignored, every other field is as for zero_step.
+ * No cudaMalloc, cudaFree or other allocating call is made.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) and
+ * caches it; make that first call before any stream capture.  All calls share
+ * the one array: calls whose kernels overlap on the GPU (several streams or
+ * threads at once) race on it and must be serialised by the caller.  Each
+ * step overwrites the array before reading it, so stale contents are harmless.
+ * ZERO_EINVAL: as zero_step, or a plan whose scratch would exceed the static
+ * array (the message says so).  ZERO_ECUDA: the address lookup or a launch
+ * failed. */
+zero_status_t zero_step_noalloc(const zero_plan_t *plan, const zero_bufs_t *bufs,
+                                const zero_adam_t *adam, uint64_t t, void *stream);
+
 /* Stage 3: materialise unit `unit` -- copy the Nd owners' bf16 slices of it,
  * in rank order, into full_layer[0 .. len_u) (padding dropped) -- and mark
  * it live.  Source: [MM] glossary "临时物化" and "all-gather" (shards are

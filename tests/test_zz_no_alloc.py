@@ -1,0 +1,59 @@
+"""zero_step_noalloc() gives the same step as zero_step().
+
+zero_step_noalloc() serves callers that cannot allocate device memory -- for
+example a runtime whose device memory is all handed out by its own pool up
+front, or a plain C caller without an allocator: instead of a caller-provided
+workspace, the gradient-norm / overflow scratch is the library's own static
+device array.  This test calls it through the C ABI twice in a row and
+checks every output against zero_step() with a caller-provided workspace on
+the same inputs.  The file is named to run last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+import zero_partitioned_optimizer_step_b200 as Z
+from zero_cases import (BF16_ULP, RTOL_NORM, RTOL_REDUCED, RTOL_STATE, Case, bf16_ulp_check,
+                        f32, f32_rel_check, u16)
+
+pytestmark = pytest.mark.gpu
+
+
+def test_noalloc_step_matches_zero_step_on_two_calls():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    ref = Case(1_000_003, 8, 2, 100_000, config_id=2)   # zero_step + workspace
+    new = Case(1_000_003, 8, 2, 100_000, config_id=2)   # zero_step_noalloc
+    L = Z.lib()
+    for t in (1, 2):
+        G = ref.grads(t)
+        ref.run_gpu(G, t)
+        bufs = Z.make_bufs(new.lp, G, new.w, new.m, new.v, new.params, reduced_grad=new.red,
+                           grad_norm_sq=new.norm, overflow=new.ovf)
+        adam = Z.make_adam(new.adam)
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        before = torch.cuda.memory_allocated()
+        st = L.zero_step_noalloc(new.lp.handle, ctypes.byref(bufs), ctypes.byref(adam), t, stream)
+        assert st == Z.ZERO_OK, L.zero_last_error().decode()
+        torch.cuda.synchronize()
+        assert torch.cuda.memory_allocated() == before
+        f32_rel_check(f32(new.w), f32(ref.w), RTOL_STATE, "master")
+        f32_rel_check(f32(new.m), f32(ref.m), RTOL_STATE, "exp_avg")
+        f32_rel_check(f32(new.v), f32(ref.v), RTOL_STATE, "exp_avg_sq")
+        f32_rel_check(f32(new.red), f32(ref.red), RTOL_REDUCED, "reduced")
+        bf16_ulp_check(u16(new.params), u16(ref.params), BF16_ULP, "params")
+        n_ref, n_new = ref.norm.item(), new.norm.item()
+        assert abs(n_new - n_ref) <= RTOL_NORM * n_ref
+        assert int(new.ovf.item()) == int(ref.ovf.item()) == 0
+
+
+def test_noalloc_rejects_bad_arguments():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    c = Case(4096, 4, 2, 1024, config_id=2)
+    G = c.grads(1)
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_step_noalloc(c.lp, G, c.w, c.m, c.v, c.params, c.adam, 0,
+                            grad_norm_sq=c.norm, overflow=c.ovf)
+    assert e.value.status == Z.ZERO_EINVAL

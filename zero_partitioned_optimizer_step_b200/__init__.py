@@ -89,6 +89,8 @@ def lib():
         L.zero_plan_query.argtypes = [vp, ctypes.c_int, u64, ctypes.POINTER(u64)]
         L.zero_step.restype = st
         L.zero_step.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam), u64, vp]
+        L.zero_step_noalloc.restype = st
+        L.zero_step_noalloc.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam), u64, vp]
         L.zero_step_buckets.restype = st
         L.zero_step_buckets.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam),
                                         u64, u64, u64, vp]
@@ -280,6 +282,17 @@ def zero_step(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t, stream=
     b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
     _check(lib().zero_step(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
                            int(t), _stream(stream)))
+
+
+def zero_step_noalloc(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t, stream=None,
+                      **kw):
+    """zero_step without a workspace argument: the norm/overflow scratch is the
+    library's own static device array (for callers that cannot allocate)."""
+    if "workspace" in kw:
+        raise ValueError("zero_step_noalloc takes no workspace")
+    b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
+    _check(lib().zero_step_noalloc(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
+                                   int(t), _stream(stream)))
 
 
 def zero_step_buckets(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t,

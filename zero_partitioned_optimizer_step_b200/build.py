@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libzero.so")
-SOURCES = [os.path.join(CSRC, f) for f in ("zero_plan.cpp", "zero_step.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("zero_plan.cpp", "zero_step.cu", "zero_noalloc.cu")]
 HEADERS = [os.path.join(CSRC, "zero_internal.h"), os.path.join(ROOT, "include", "zero.h")]
 
 NVCC_FLAGS = [
