@@ -38,8 +38,18 @@ if ROOT not in sys.path:
 METRIC = "Gparams/s per ZeRO step (RS+Adam+AG); achieved HBM GB/s vs B200 peak"
 UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
-K1_PROFILE = os.path.join(ROOT, "profiles", "k_step_vec8_gpt2_small_nd8.md")
-K1_SOURCE = os.path.join(ROOT, "zero_partitioned_optimizer_step_b200", "csrc", "zero_step.cu")
+K1_PROFILE = os.path.join(ROOT, "profiles", "k_step_tma_gpt2_small_nd8.md")
+K1_SOURCES = [os.path.join(ROOT, "zero_partitioned_optimizer_step_b200", "csrc", f)
+              for f in ("zero_step.cu", "zero_tma.cuh", "zero_device.cuh")]
+
+
+def kernel_source_hash():
+    """First 16 hex digits of sha256 over the step kernels' sources."""
+    h = hashlib.sha256()
+    for f in K1_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def parse_args():
@@ -87,7 +97,7 @@ def k1_traffic_per_elem():
     summary, if it was taken on the current kernel source (else None)."""
     try:
         txt = open(K1_PROFILE, encoding="utf-8").read()
-        src_hash = hashlib.sha256(open(K1_SOURCE, "rb").read()).hexdigest()[:16]
+        src_hash = kernel_source_hash()
         m = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
         b = re.search(r"dram_bytes_per_element:\s*([0-9.eE+-]+)", txt)
         if m and b and m.group(1) == src_hash:
@@ -208,6 +218,14 @@ class Workload:
         self.elems = self.S if owner >= 0 else self.psi_pad
         self.params_per_step = (min(max(cfg["psi"] - owner * self.S, 0), self.S)
                                 if owner >= 0 else cfg["psi"])
+        self.nb = self.lp.n_buckets
+
+    def rebucket(self, bucket_elems):
+        """Same buffers, a new plan with another bucket size."""
+        cfg = self.cfg
+        self.cfg = dict(cfg, bucket_elems=bucket_elems)
+        self.lp = self.Z.zero_plan(cfg["psi"], cfg["nd"], cfg["stage"], bucket_elems,
+                                   unit_elems=cfg["units"])
         self.nb = self.lp.n_buckets
 
     def bucket_elems(self, b):
@@ -404,7 +422,8 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
     achieved = k1_bytes / k1_time / 1e9
     n_launch = args.steps * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
     tr = k1_traffic_per_elem() if (args.config == "c2" and args.psi is None) else None
-    roof = {"kernel": "k_step_vec8 (fused reduce-scatter + Adam + all-gather, one bucket)",
+    roof = {"kernel": "k_step_tma (fused reduce-scatter + Adam + all-gather, one bucket; "
+                      "bulk-copy ring)",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
             "traffic": None if tr is None else tr * k1_elems / n_launch,
@@ -434,6 +453,54 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
     return out
 
 
+def run_sweep(args, rank, world, dist):
+    """The bucket-size sweep (5e8 params): for each Nd one set of buffers, then
+    every bucket size from 1 MB to 512 MB of one rank's bf16 gradient."""
+    import torch
+    from zero_partitioned_optimizer_step_b200.configs import c5_config
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    with open(args.sweep, "w") as f:
+        for nd in (2, 4, 8, 16, 64):
+            wl = Workload(c5_config(nd, 1), dev)
+            for mb in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512):
+                wl.rebucket(mb << 19)
+                cfg = dict(wl.cfg, workload="bucket sweep psi=5e8, Nd=%d, %d MB buckets" % (nd, mb))
+                stream = torch.cuda.current_stream(dev)
+                for t in range(1, args.warmup + 1):
+                    wl.step(t, stream)
+                s0 = torch.cuda.Event(enable_timing=True)
+                s1 = torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                s0.record(stream)
+                for k in range(args.steps):          # the step as a user runs it
+                    wl.step(args.warmup + 1 + k, stream)
+                s1.record(stream)
+                torch.cuda.synchronize()
+                elapsed = s0.elapsed_time(s1) / 1e3
+                # again with an event around every bucket, for the kernel's own rate
+                events = [[torch.cuda.Event(enable_timing=True) for _ in range(wl.nb + 1)]
+                          for _ in range(args.steps)]
+                for k in range(args.steps):
+                    wl.step(args.warmup + args.steps + 1 + k, stream, events[k])
+                torch.cuda.synchronize()
+                k1_time = sum(events[k][b].elapsed_time(events[k][b + 1]) / 1e3
+                              for k in range(args.steps) for b in range(wl.nb))
+                k1_elems = args.steps * sum(wl.bucket_elems(b) for b in range(wl.nb))
+                a = argparse.Namespace(**vars(args))
+                a.config = "c5"
+                a.no_cpu_baseline = True
+                res = _report(a, cfg, wl, world, elapsed, k1_time, k1_elems, None, None)
+                res["config"]["bucket_mb"] = mb
+                f.write(json.dumps(res) + "\n")
+                f.flush()
+                print(json.dumps({"nd": nd, "mb": mb, "value": res["value"],
+                                  "step_gbs": res["hbm_gbs"], "k1_gbs": res["roofline"]["achieved"],
+                                  "k1_frac": res["roofline"]["frac"]}), flush=True)
+            del wl
+            torch.cuda.empty_cache()
+
+
 def main():
     args = parse_args()
     rank = int(os.environ.get("RANK", 0))
@@ -452,23 +519,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
         if args.sweep:
-            from zero_partitioned_optimizer_step_b200.configs import c5_config
-            with open(args.sweep, "w") as f:
-                for nd in (2, 4, 8, 16, 64):
-                    for mb in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512):
-                        a = argparse.Namespace(**vars(args))
-                        a.config = "c5"
-                        a.no_cpu_baseline = True
-                        a.no_e2e = True
-                        res = run_ours(a, c5_config(nd, mb), rank, world, dist)
-                        if res is not None:
-                            res["config"]["bucket_mb"] = mb
-                            f.write(json.dumps(res) + "\n")
-                            f.flush()
-                            print(json.dumps({"nd": nd, "mb": mb, "value": res["value"],
-                                              "hbm_gbs": res["roofline"]["achieved"]}), flush=True)
-                        import torch
-                        torch.cuda.empty_cache()
+            run_sweep(args, rank, world, dist)
             return 0
         res = run_ours(args, cfg, rank, world, dist)
         if res is not None:

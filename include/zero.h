@@ -51,7 +51,13 @@
  * faults inside a kernel are asynchronous and surface on a later CUDA call.
  *
  * Streams.  `stream` is a cudaStream_t passed as void*; NULL is the legacy
- * default stream.  Launches are asynchronous; nothing synchronises.
+ * default stream.  Launches are asynchronous; nothing synchronises except
+ * zero_stream_status().
+ *
+ * Kernels.  Aligned bucket bodies run in the bulk-copy (TMA) kernel when its
+ * shared-memory ring fits Nd rows, else in the 16-byte-vector load kernel;
+ * unaligned heads and tails in a scalar kernel.  All give identical results.
+ * The environment variable ZERO_STEP_KERNEL=ldg|tma overrides the choice.
  * Threads.  A plan may be shared by threads for zero_step*() and queries;
  * zero_gather_layer()/zero_release_layer() serialise on the plan internally.
  */
@@ -273,6 +279,14 @@ typedef enum zero_bytes_kind {
  * argument or unknown kind. */
 zero_status_t zero_bytes_moved(const zero_plan_t *plan, zero_bytes_kind_t kind,
                                uint32_t flags, uint64_t *out);
+
+/* Wait for `stream` and report device-side failures of the step kernels:
+ * ZERO_ETIMEOUT if a bounded wait inside the bulk-copy step kernel gave up
+ * since the last call (the outputs of those steps are not valid; the flag is
+ * cleared), ZERO_ECUDA if the stream reports a CUDA error, else ZERO_OK.
+ * Synchronises the stream (and reads one device word), so call it between
+ * steps, not inside a captured graph. */
+zero_status_t zero_stream_status(void *stream);
 
 /* Static text of a status code. */
 const char *zero_status_str(zero_status_t status);

@@ -20,8 +20,17 @@ def _cuda():
     torch.cuda.empty_cache()
 
 
+@pytest.fixture(params=["tma", "ldg"])
+def kernel(request, monkeypatch):
+    """Run the test with the bulk-copy (TMA) kernel and with the 16-byte
+    vector-load kernel for aligned bucket bodies."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", request.param)
+    yield request.param
+    Z.zero_stream_status()
+
+
 @pytest.mark.parametrize("stage", [0, 1, 2, 3])
-def test_toy_four_ranks_bit_exact(stage):
+def test_toy_four_ranks_bit_exact(stage, kernel):
     """The four-rank A/B/C/D toy, 3 steps: every output bit-identical to the
     oracle (which is itself pinned to equal replicated Adam)."""
     c = Case(65_536, 4, stage, 16_384, sigma=0.01, config_id=1)
@@ -59,7 +68,7 @@ RAGGED = [
 
 
 @pytest.mark.parametrize("psi,nd,stage,bucket,align,units", RAGGED)
-def test_ragged_shapes(psi, nd, stage, bucket, align, units):
+def test_ragged_shapes(psi, nd, stage, bucket, align, units, kernel):
     """Odd sizes, scalar and vector paths, bucket heads and tails, several
     units (owner storage != logical order), Nd from 1 to 64."""
     c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=7)
@@ -68,7 +77,7 @@ def test_ragged_shapes(psi, nd, stage, bucket, align, units):
 
 
 @pytest.mark.parametrize("owner", [0, 5, 63])
-def test_owner_view(owner):
+def test_owner_view(owner, kernel):
     """One owner's shard with its slices of all 64 ranks' gradients."""
     c = Case(1_000_000, 64, 2, 100_000, owner_view=owner, config_id=4)
     for t in (1, 2, 3):
@@ -76,13 +85,13 @@ def test_owner_view(owner):
         assert all(v == 0 for v in diff.values()), diff
 
 
-def test_owner_view_multi_unit():
+def test_owner_view_multi_unit(kernel):
     c = Case(300_001, 16, 3, 20_000, units=[100_000, 1, 200_000], owner_view=9, config_id=4)
     for t in (1, 2):
         c.step_and_compare(t)
 
 
-def test_bucket_calls_compose():
+def test_bucket_calls_compose(kernel):
     """zero_step_buckets over pieces == zero_step in one call, norm included."""
     a = Case(500_000, 8, 2, 40_000, config_id=2)
     b = Case(500_000, 8, 2, 40_000, config_id=2)
@@ -102,7 +111,7 @@ def test_bucket_calls_compose():
         assert a.norm.item() == b.norm.item()
 
 
-def test_norm_and_overflow_flag():
+def test_norm_and_overflow_flag(kernel):
     c = Case(200_000, 4, 2, 50_000, config_id=6)
     G = c.grads(1)
     G[1, 123] = float("inf")
@@ -117,7 +126,7 @@ def test_norm_and_overflow_flag():
     assert int(c.ovf.item()) == 0
 
 
-def test_norm_is_deterministic():
+def test_norm_is_deterministic(kernel):
     c = Case(300_000, 8, 2, 30_000, config_id=6, with_reduced=False)
     G = c.grads(1)
     vals = set()
@@ -128,7 +137,7 @@ def test_norm_is_deterministic():
     assert len(vals) == 1
 
 
-def test_zero_gradient_keeps_state_and_padding():
+def test_zero_gradient_keeps_state_and_padding(kernel):
     c = Case(10_001, 8, 2, 4096, config_id=5)
     G = torch.zeros((8, c.op.psi_pad), dtype=torch.bfloat16, device="cuda")
     w0 = f32(c.w).copy()
@@ -203,3 +212,24 @@ def test_library_errors_on_device_calls():
         Z.zero_step(c.lp, G[:, 1:], c.w, c.m, c.v, c.params, c.adam, 1)   # misaligned
     with pytest.raises(ValueError):
         Z.zero_step(c.lp, G.float(), c.w, c.m, c.v, c.params, c.adam, 1)
+
+
+def test_kernels_agree_bitwise_large_nd():
+    """Nd = 64 and Nd = 100 (ring of 3 and 2 stages): both vector kernels give
+    the same bits."""
+    import os
+    for nd in (64, 100):
+        outs = []
+        for k in ("tma", "ldg"):
+            os.environ["ZERO_STEP_KERNEL"] = k
+            try:
+                c = Case(300_000, nd, 2, 1 << 20, config_id=9, with_reduced=True)
+                G = c.grads(1)
+                c.run_gpu(G, 1)
+                Z.zero_stream_status()
+                outs.append([f32(c.w), f32(c.m), f32(c.v), f32(c.red), u16(c.params), c.norm.item()])
+            finally:
+                del os.environ["ZERO_STEP_KERNEL"]
+        for x, y in zip(outs[0][:5], outs[1][:5]):
+            assert np.array_equal(x, y)
+        assert outs[0][5] == pytest.approx(outs[1][5], rel=1e-12)

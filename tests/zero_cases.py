@@ -147,7 +147,7 @@ class Case:
         Gh = u16(G)
         self.run_gpu(G, t)
         norm, bad = self.run_oracle(Gh, t)
-        torch.cuda.synchronize()
+        Z.zero_stream_status()          # synchronises; raises if a wait gave up
         return self.compare(norm, bad)
 
     def compare(self, norm, bad):

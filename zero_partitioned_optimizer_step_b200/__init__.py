@@ -100,6 +100,8 @@ def lib():
         L.zero_release_layer.argtypes = [vp, ctypes.c_uint32]
         L.zero_bytes_moved.restype = st
         L.zero_bytes_moved.argtypes = [vp, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(u64)]
+        L.zero_stream_status.restype = st
+        L.zero_stream_status.argtypes = [vp]
         L.zero_status_str.restype = ctypes.c_char_p
         L.zero_status_str.argtypes = [ctypes.c_int]
         L.zero_last_error.restype = ctypes.c_char_p
@@ -309,6 +311,12 @@ def zero_gather_layer(plan, unit, owner_params, full_layer, stream=None):
                                    _ptr(owner_params, torch.bfloat16, "owner_params"),
                                    _ptr(full_layer, torch.bfloat16, "full_layer"),
                                    _stream(stream)))
+
+
+def zero_stream_status(stream=None):
+    """Synchronise the stream; raise ZeroError(ZERO_ETIMEOUT) if a bounded
+    wait in the bulk-copy kernel gave up since the last check."""
+    _check(lib().zero_stream_status(_stream(stream)))
 
 
 def workspace_for(plan, device="cuda"):

@@ -1,0 +1,80 @@
+// Device-side definitions shared by the step kernels: the launch arguments
+// of one bucket, the Adam constants, bf16 packing and the per-element update.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace zero_dev {
+
+constexpr int kThreads = 256;
+constexpr int kRB = 4;    // gradient rows in flight per thread
+constexpr int kMinB = 2;  // CTAs per SM the vector kernel is sized for
+
+struct AdamConsts {
+    float grad_scale, beta1, beta2, eps, omb1, omb2, step, ibc2;
+};
+
+// One launch: the unit-local element range [j0, j1) of one bucket.
+// Element j reads gradients at  g_base + j           (+ r*grad_stride),
+// state at                      s_base + j + o*jump,
+// parameters at                 p_base + j + o*p_jump (+ row*param_stride),
+// where o = j / shard is the owner (used only when the unit is one of several,
+// so that owner storage and logical order differ).
+struct StepArgs {
+    const uint16_t *grads;
+    uint64_t grad_stride;
+    float *w, *m, *v, *red;
+    uint16_t *params;
+    uint64_t param_stride;
+    uint32_t n_prow;
+    uint32_t nd;
+    int64_t g_base, s_base, p_base;
+    uint64_t shard, jump, p_jump;
+    uint64_t j0, j1;
+    AdamConsts c;
+    double *ws_norm;
+    uint32_t *ws_bad;
+    int ws_mode;  // 0: no norm; 1: add this launch's per-CTA partials to the slots
+};
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ void unpack8(const uint4 x, float f[8]) {
+    f[0] = bf16lo(x.x); f[1] = bf16hi(x.x);
+    f[2] = bf16lo(x.y); f[3] = bf16hi(x.y);
+    f[4] = bf16lo(x.z); f[5] = bf16hi(x.z);
+    f[6] = bf16lo(x.w); f[7] = bf16hi(x.w);
+}
+
+__device__ __forceinline__ void add8(float s[8], const uint4 x) {
+    float f[8];
+    unpack8(x, f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[e] = __fadd_rn(s[e], f[e]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ bool not_finite(float x) {
+    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+// Textbook Adam on one element, every operation rounded to nearest.
+__device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w, float &m,
+                                      float &v) {
+    const float g = __fmul_rn(g_sum, c.grad_scale);
+    const float m_new = __fadd_rn(__fmul_rn(c.beta1, m), __fmul_rn(c.omb1, g));
+    const float v_new = __fadd_rn(__fmul_rn(c.beta2, v), __fmul_rn(__fmul_rn(c.omb2, g), g));
+    const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v_new), c.ibc2), c.eps);
+    const float delta = __fmul_rn(c.step, __fdiv_rn(m_new, denom));
+    w = __fsub_rn(w, delta);
+    m = m_new;
+    v = v_new;
+}
+
+}  // namespace zero_dev

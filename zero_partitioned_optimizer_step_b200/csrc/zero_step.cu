@@ -38,86 +38,23 @@
 #include <cstdint>
 #include <map>
 #include <mutex>
+#include <cstdlib>
+#include <cstring>
 #include <string>
 
+#include "zero_device.cuh"
+#include "zero_tma.cuh"
 #include "zero_internal.h"
 
 using zero_detail::set_error;
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRB = 4;    // gradient rows in flight per thread
-constexpr int kMinB = 2;  // CTAs per SM the vector kernel is sized for
+using namespace zero_dev;
 
-struct AdamConsts {
-    float grad_scale, beta1, beta2, eps, omb1, omb2, step, ibc2;
-};
-
-// One launch: the unit-local element range [j0, j1) of one bucket.
-// Element j reads gradients at  g_base + j           (+ r*grad_stride),
-// state at                      s_base + j + o*jump,
-// parameters at                 p_base + j + o*p_jump (+ row*param_stride),
-// where o = j / shard is the owner (used only when the unit is one of several,
-// so that owner storage and logical order differ).
-struct StepArgs {
-    const uint16_t *grads;
-    uint64_t grad_stride;
-    float *w, *m, *v, *red;
-    uint16_t *params;
-    uint64_t param_stride;
-    uint32_t n_prow;
-    uint32_t nd;
-    int64_t g_base, s_base, p_base;
-    uint64_t shard, jump, p_jump;
-    uint64_t j0, j1;
-    AdamConsts c;
-    double *ws_norm;
-    uint32_t *ws_bad;
-    int ws_mode;  // 0: no norm; 1: store this launch's partials; 2: add them
-};
-
-__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ void unpack8(const uint4 x, float f[8]) {
-    f[0] = bf16lo(x.x); f[1] = bf16hi(x.x);
-    f[2] = bf16lo(x.y); f[3] = bf16hi(x.y);
-    f[4] = bf16lo(x.z); f[5] = bf16hi(x.z);
-    f[6] = bf16lo(x.w); f[7] = bf16hi(x.w);
-}
-
-__device__ __forceinline__ void add8(float s[8], const uint4 x) {
-    float f[8];
-    unpack8(x, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = __fadd_rn(s[e], f[e]);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ bool not_finite(float x) {
-    return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
-}
-
-// Textbook Adam on one element, every operation rounded to nearest.
-__device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w, float &m,
-                                      float &v) {
-    const float g = __fmul_rn(g_sum, c.grad_scale);
-    const float m_new = __fadd_rn(__fmul_rn(c.beta1, m), __fmul_rn(c.omb1, g));
-    const float v_new = __fadd_rn(__fmul_rn(c.beta2, v), __fmul_rn(__fmul_rn(c.omb2, g), g));
-    const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v_new), c.ibc2), c.eps);
-    const float delta = __fmul_rn(c.step, __fdiv_rn(m_new, denom));
-    w = __fsub_rn(w, delta);
-    m = m_new;
-    v = v_new;
-}
-
-// Per-CTA partials of the gradient-norm / overflow reduction (fixed order,
-// so the reported norm is the same on every run of the same launch shape).
+// Per-CTA partials of the gradient-norm / overflow reduction, added to slot
+// blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
+// so the reported norm is the same on every run of the same launch shapes.
 __device__ __forceinline__ void block_partials(double acc, uint32_t bad, const StepArgs &a) {
     __shared__ double sd[kThreads / 32];
     __shared__ uint32_t sb[kThreads / 32];
@@ -139,13 +76,8 @@ __device__ __forceinline__ void block_partials(double acc, uint32_t bad, const S
             t += sd[i];
             b += sb[i];
         }
-        if (a.ws_mode == 1) {
-            a.ws_norm[blockIdx.x] = t;
-            a.ws_bad[blockIdx.x] = b;
-        } else {
-            a.ws_norm[blockIdx.x] += t;
-            a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
-        }
+        a.ws_norm[blockIdx.x] += t;
+        a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
     }
 }
 
@@ -336,30 +268,122 @@ __global__ void __launch_bounds__(kThreads) k_gather(const uint16_t *src, uint64
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Grid of the step kernels on the current device: SM count x resident CTAs
-// of the vector kernel, capped at the workspace's slot count.  Cached per
-// device; all launches of a step use it, so the norm slots line up.
-zero_status_t device_grid(uint32_t *grid) {
+// Launch shapes of the step kernels on one device, computed once per device:
+// the persistent grid of the vector kernel (SM count x resident CTAs, capped
+// at the norm workspace's slot count), the SM count for the bulk-copy kernel
+// (one CTA per SM: its ring takes most of shared memory), and the dynamic
+// shared memory the bulk-copy kernel may use.
+struct DeviceShapes {
+    uint32_t grid_ldg = 0;
+    uint32_t sms = 0;
+    uint32_t tma_smem = 0;
+};
+
+zero_status_t device_shapes(DeviceShapes *out) {
     static std::mutex mu;
-    static std::map<int, uint32_t> cache;
+    static std::map<int, DeviceShapes> cache;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
     std::lock_guard<std::mutex> g(mu);
     auto it = cache.find(dev);
     if (it != cache.end()) {
-        *grid = it->second;
+        *out = it->second;
         return ZERO_OK;
     }
-    int sms = 0, occ = 0;
+    int sms = 0, occ = 0, optin = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_vec8<false, kRB, kMinB>, kThreads, 0);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_vec8<false, kRB, kMinB>, kThreads, 0);
+    cudaFuncAttributes fa{};
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, zero_tma::k_step_tma<true, 2>);
+    DeviceShapes d;
+    d.sms = uint32_t(std::max(1, sms));
+    d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
+    const int64_t budget = int64_t(optin) - int64_t(fa.sharedSizeBytes) - 256;
+    d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
+    if (d.tma_smem > 0) {
+        const void *fns[] = {reinterpret_cast<const void *>(zero_tma::k_step_tma<true, 1>),
+                             reinterpret_cast<const void *>(zero_tma::k_step_tma<false, 1>),
+                             reinterpret_cast<const void *>(zero_tma::k_step_tma<true, 2>),
+                             reinterpret_cast<const void *>(zero_tma::k_step_tma<false, 2>)};
+        for (const void *f : fns)
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
+    }
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("device query: ") + cudaGetErrorString(e));
-    uint32_t gsz = uint32_t(std::max(1, sms) * std::max(1, occ));
-    gsz = std::min(gsz, zero_detail::kMaxSlots);
-    cache[dev] = gsz;
-    *grid = gsz;
+    cache[dev] = d;
+    *out = d;
     return ZERO_OK;
+}
+
+uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
+
+// Shared-memory ring of the bulk-copy kernel for Nd gradient rows.  Each
+// tile pays a fixed synchronisation latency, so tiles are large; two consumer
+// groups help where a tile is cheap to compute.  Shapes measured best on B200
+// at 64 MB buckets (5e8 params):
+//   Nd <= 4: 2 groups, 2048-element tiles, 4 stages
+//   Nd <= 8: 1 group, 2048, 3       Nd <= 16: 2 groups, 2048, 2
+//   Nd <= 32: 2 groups, 1024, 2     Nd <= 64: 1 group, 512, 3
+// Beyond 64 ranks (or when the shape does not fit) the 16-byte-load kernel is
+// used.  With two groups the stage count is even (each group owns half the
+// stages).  ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS override the
+// shape (tuning; a tile must be a positive multiple of 256).
+zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t groups) {
+    zero_tma::Ring q;
+    q.tile = uint32_t(t);
+    q.off_w = align128(uint64_t(nd) * t * 2);
+    q.off_m = q.off_w + align128(4 * t);
+    q.off_v = q.off_m + align128(4 * t);
+    q.stage_bytes = q.off_v + align128(4 * t);
+    q.stages = stages;
+    q.groups = groups;
+    return q;
+}
+
+bool choose_ring(uint32_t nd, uint32_t budget, zero_tma::Ring *r) {
+    long force_t = 0, force_s = 0, force_g = 0;
+    if (const char *e = std::getenv("ZERO_TMA_TILE")) force_t = std::strtol(e, nullptr, 10);
+    if (const char *e = std::getenv("ZERO_TMA_STAGES")) force_s = std::strtol(e, nullptr, 10);
+    if (const char *e = std::getenv("ZERO_TMA_GROUPS")) force_g = std::strtol(e, nullptr, 10);
+    uint32_t groups, stages;
+    uint64_t tile;
+    if (force_t >= 256 && force_t % 256 == 0 && force_t <= 16384) {
+        tile = uint64_t(force_t);
+        groups = force_g == 2 ? 2 : 1;
+        stages = force_s >= 2 ? uint32_t(std::min<long>(force_s, zero_tma::kMaxStages)) : zero_tma::kMaxStages;
+    } else if (nd <= 4) {
+        groups = 2, tile = 2048, stages = 4;
+    } else if (nd <= 8) {
+        groups = 1, tile = 2048, stages = 3;
+    } else if (nd <= 16) {
+        groups = 2, tile = 2048, stages = 2;
+    } else if (nd <= 32) {
+        groups = 2, tile = 1024, stages = 2;
+    } else if (nd <= 64) {
+        groups = 1, tile = 512, stages = 3;
+    } else {
+        return false;
+    }
+    zero_tma::Ring q = ring_for(nd, tile, 0, groups);
+    uint64_t ns = std::min<uint64_t>(budget / q.stage_bytes, stages);
+    ns -= ns % groups;  // every stage belongs to one group
+    if (ns < 2) return false;
+    q.stages = uint32_t(ns);
+    *r = q;
+    return true;
+}
+
+// ZERO_STEP_KERNEL=ldg|tma picks the vector kernel for aligned bucket bodies
+// (default: the bulk-copy kernel whenever its ring fits).
+int kernel_choice() {
+    const char *s = std::getenv("ZERO_STEP_KERNEL");
+    if (!s) return 0;
+    if (std::strcmp(s, "ldg") == 0) return 1;
+    if (std::strcmp(s, "tma") == 0) return 2;
+    return 0;
 }
 
 AdamConsts make_consts(const zero_adam_t &a, uint64_t t) {
@@ -387,10 +411,11 @@ zero_status_t check_launch(const char *what) {
 bool mult8(int64_t x) { return (uint64_t(x) & 7u) == 0; }
 
 struct Launcher {
-    uint32_t grid;
+    DeviceShapes shapes;
     cudaStream_t stream;
-    bool first = true;   // next launch stores (not adds) its norm partials
     bool want_ws = false;
+    bool use_tma = false;
+    zero_tma::Ring ring{};
     uint32_t launches = 0;
 
     zero_status_t run(StepArgs a, bool owner_map, bool vec_ok) {
@@ -400,16 +425,27 @@ struct Launcher {
             StepArgs b = a;
             b.j0 = j0;
             b.j1 = j1;
-            b.ws_mode = want_ws ? (first ? 1 : 2) : 0;
-            if (vec) {
-                if (owner_map)
-                    k_step_vec8<true, kRB, kMinB><<<grid, kThreads, 0, stream>>>(b);
+            b.ws_mode = want_ws ? 1 : 0;
+            if (vec && use_tma) {
+                const uint64_t tiles = (j1 - j0 + ring.tile - 1) / ring.tile;
+                const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
+                const size_t smem = size_t(ring.stages) * ring.stage_bytes;
+                if (owner_map && ring.groups == 2)
+                    zero_tma::k_step_tma<true, 2><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
+                else if (owner_map)
+                    zero_tma::k_step_tma<true, 1><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
+                else if (ring.groups == 2)
+                    zero_tma::k_step_tma<false, 2><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
                 else
-                    k_step_vec8<false, kRB, kMinB><<<grid, kThreads, 0, stream>>>(b);
+                    zero_tma::k_step_tma<false, 1><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
+            } else if (vec) {
+                if (owner_map)
+                    k_step_vec8<true, kRB, kMinB><<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
+                else
+                    k_step_vec8<false, kRB, kMinB><<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
             } else {
-                k_step_scalar<<<grid, kThreads, 0, stream>>>(b);
+                k_step_scalar<<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
             }
-            first = false;
             ++launches;
             return check_launch("zero_step kernel launch");
         };
@@ -465,8 +501,8 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     cudaError_t pre = cudaPeekAtLastError();
     if (pre != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_step: ") + cudaGetErrorString(pre));
-    uint32_t grid = 0;
-    st = device_grid(&grid);
+    DeviceShapes shapes;
+    st = device_shapes(&shapes);
     if (st != ZERO_OK) return st;
 
     const bool owner = b->owner_view >= 0;
@@ -490,10 +526,17 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     a.ws_bad = reinterpret_cast<uint32_t *>(ws + 8ull * zero_detail::kMaxSlots);
 
     Launcher L;
-    L.grid = grid;
+    L.shapes = shapes;
     L.stream = static_cast<cudaStream_t>(stream_);
     L.want_ws = b->grad_norm_sq || b->overflow;
-    L.first = (first == 0);
+    const int choice = kernel_choice();
+    L.use_tma = choice != 1 && choose_ring(p->nd, shapes.tma_smem, &L.ring);
+    if (L.want_ws && first == 0) {
+        // the step's first call zeroes the per-CTA norm slots
+        cudaError_t e = cudaMemsetAsync(b->workspace, 0, zero_detail::kWorkspaceBytes, L.stream);
+        if (e != cudaSuccess)
+            return set_error(ZERO_ECUDA, std::string("zero_step workspace reset: ") + cudaGetErrorString(e));
+    }
 
     const bool strides_ok = (b->grad_stride & 7u) == 0 && (!replicas || (b->param_stride & 7u) == 0);
     for (uint64_t bk = first; bk < first + count; ++bk) {
@@ -528,7 +571,8 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
         if (st != ZERO_OK) return st;
     }
     if (L.want_ws && first + count == p->n_buckets && count > 0) {
-        k_finalize<<<1, kThreads, 0, L.stream>>>(a.ws_norm, a.ws_bad, grid, b->grad_norm_sq, b->overflow);
+        k_finalize<<<1, kThreads, 0, L.stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots, b->grad_norm_sq,
+                                                 b->overflow);
         st = check_launch("zero_step finalize launch");
         if (st != ZERO_OK) return st;
     }
@@ -562,9 +606,10 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
     if (pre != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_gather_layer: ") +
                                          cudaGetErrorString(pre));
-    uint32_t grid = 0;
-    zero_status_t st = device_grid(&grid);
+    DeviceShapes shapes;
+    zero_status_t st = device_shapes(&shapes);
     if (st != ZERO_OK) return st;
+    const uint32_t grid = shapes.grid_ldg;
     const uint64_t s_u = p->unit_shard[unit], off = p->unit_offset[unit], len = p->unit_len[unit];
     const int vec_ok = ((p->S | off | s_u) & 7u) == 0;
     const uint32_t cpo = std::max<uint32_t>(1, grid / p->nd);
@@ -580,5 +625,24 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
     p->live_bytes += 2 * len;
     p->peak_live = std::max(p->peak_live, p->n_live);
     p->peak_live_bytes = std::max(p->peak_live_bytes, p->live_bytes);
+    return ZERO_OK;
+}
+
+ZERO_API zero_status_t zero_stream_status(void *stream) {
+    zero_detail::clear_error();
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("zero_stream_status: ") + cudaGetErrorString(e));
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, zero_tma::g_wait_error, sizeof v);
+    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("zero_stream_status: ") + cudaGetErrorString(e));
+    if (v) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(zero_tma::g_wait_error, &zero, sizeof zero);
+        return set_error(ZERO_ETIMEOUT,
+                         v == 2 ? "zero_stream_status: the bulk-copy step kernel found a stage holding the wrong "
+                                  "tile and gave up; the outputs of the steps since the last check are not valid"
+                                : "zero_stream_status: a bounded wait in the bulk-copy step kernel gave up; the "
+                                  "outputs of the steps since the last check are not valid");
+    }
     return ZERO_OK;
 }

@@ -1,0 +1,337 @@
+// K1, bulk-copy path (sm_100a): the fused reduce-scatter + Adam + all-gather
+// of one bucket with its operands staged through a shared-memory ring by the
+// Tensor Memory Accelerator's 1-D bulk copies.
+//
+// Warp 0 is the producer.  Per tile of `tile` elements it issues one
+// cp.async.bulk per gradient row (Nd rows, spread over its lanes) and one per
+// state array and owner segment, all completing on the stage's `full`
+// mbarrier.  Warps 1..8 are consumers: they read the stage from shared memory,
+// sum the rows in rank order, run Adam, and write w, m, v and the bf16
+// parameters (every replica row, or the owner shard) straight from registers
+// with 16-byte streaming stores.  The stage is released through its `empty`
+// mbarrier as soon as the consumers have read it, so the producer keeps
+// (stages - 1) tiles of loads in flight per SM: registers no longer bound the
+// bytes in flight.  No multicast is used.
+//
+// Every wait is bounded (kWaitLimitNs of %globaltimer).  A thread that gives
+// up sets the CTA's abort flag and the device error word g_wait_error; the
+// consumers leave the loop together (the decision is an OR-reduction over a
+// barrier, so no consumer is left alone at a barrier), the producer waits a
+// bounded time for the loads it issued, and the kernel returns.
+// zero_stream_status() reports the error word.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "zero_device.cuh"
+
+namespace zero_tma {
+
+using zero_dev::AdamConsts;
+using zero_dev::StepArgs;
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;
+constexpr int kThreads = 32 + kConsumers;  // warp 0 produces
+// Consumers form GROUPS groups (a template parameter, 1 or 2) that take the
+// CTA's tiles in turn.  Tile k goes to stage k % stages and to group
+// k % GROUPS; the host makes `stages` a multiple of GROUPS, so every stage
+// belongs to one group, which waits for its uses strictly in order.  (A group
+// waiting on a stage that another group is still using could see the parity
+// of an older, unfinished phase as "done": mbarrier parity waits only
+// distinguish the current phase from the one before it.)
+constexpr int kMaxStages = 8;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Shared-memory ring chosen on the host.  A stage holds Nd gradient rows of
+// `tile` bf16 at offset 0, then w, m, v (fp32).
+struct Ring {
+    uint32_t tile;
+    uint32_t stages;  // a multiple of groups
+    uint32_t groups;  // consumer groups the kernel was instantiated with
+    uint32_t stage_bytes;
+    uint32_t off_w, off_m, off_v;
+};
+
+// Device error word: 1 once a bounded wait has given up, 2 if a consumer found
+// a stage holding another tile than the one it expected.
+__device__ int g_wait_error;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `bar` with the given parity.  Gives up (returning
+// false) when the CTA's abort flag is raised, or after kWaitLimitNs, in which
+// case it raises the abort flag and the device error word.
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicExch(&g_wait_error, 1);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Named barrier `id` over `count` threads, returning the OR of `v` over them
+// (the same value in every participating thread).  Ids: 1 + group for a
+// consumer group, 1 + GROUPS for all consumers.
+__device__ __forceinline__ bool barrier_or(uint32_t id, uint32_t count, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+// Calls f(j, count, state_shift, param_shift) for each piece of [jb, je) that
+// has one owner: the state of element j sits at s_base + j + state_shift.
+template <bool OWNER_MAP, typename F>
+__device__ __forceinline__ void for_each_segment(const StepArgs &a, uint64_t jb, uint64_t je, F f) {
+    if (!OWNER_MAP) {
+        f(jb, je - jb, uint64_t(0), uint64_t(0));
+        return;
+    }
+    uint64_t o = jb / a.shard;
+    uint64_t j = jb;
+    while (j < je) {
+        const uint64_t e = min(je, (o + 1) * a.shard);
+        f(j, e - j, o * a.jump, o * a.p_jump);
+        j = e;
+        ++o;
+    }
+}
+
+__device__ __forceinline__ uint4 lds128(const unsigned char *p) {
+    return *reinterpret_cast<const uint4 *>(p);
+}
+
+template <bool OWNER_MAP, int GROUPS>
+__global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, const Ring ring) {
+    constexpr uint32_t kGroupThreads = kConsumers / GROUPS;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full_bar[kMaxStages];
+    __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
+    __shared__ uint64_t stage_tile[kMaxStages];  // tile a stage was filled with
+    __shared__ int s_abort;
+    __shared__ double s_norm[kConsumerWarps];
+    __shared__ uint32_t s_bad[kConsumerWarps];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t T = ring.tile;
+    const uint32_t NS = ring.stages;
+    const uint64_t n_tiles = (a.j1 - a.j0 + T - 1) / T;
+
+    if (threadIdx.x == 0) {
+        for (uint32_t s = 0; s < NS; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        s_abort = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    volatile int *abort_flag = &s_abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        uint32_t k = 0;
+        for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
+            const uint32_t s = k % NS;
+            if (k >= NS) {
+                int ok = 1;
+                if (lane == 0) ok = mbar_wait(&empty_bar[s], ((k / NS) - 1) & 1u, abort_flag);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
+            const uint64_t jb = a.j0 + tile * T;
+            const uint64_t je = min(jb + T, a.j1);
+            const uint32_t n = uint32_t(je - jb);
+            unsigned char *st = smem + size_t(s) * ring.stage_bytes;
+            if (lane == 0) {
+                stage_tile[s] = tile;  // published by the arrive below (release)
+                mbar_arrive_expect_tx(&full_bar[s], n * (2u * a.nd + 12u));
+            }
+            __syncwarp();
+            const uint16_t *g = a.grads + uint64_t(a.g_base + int64_t(jb));
+            for (uint32_t r = lane; r < a.nd; r += 32)
+                bulk_load(st + size_t(r) * T * 2, g + uint64_t(r) * a.grad_stride, n * 2u, &full_bar[s]);
+            if (lane == 0) {
+                for_each_segment<OWNER_MAP>(a, jb, je, [&](uint64_t js, uint64_t cnt, uint64_t so, uint64_t) {
+                    const uint64_t off = js - jb;
+                    const uint64_t si = uint64_t(a.s_base + int64_t(js)) + so;
+                    bulk_load(st + ring.off_w + off * 4, a.w + si, uint32_t(cnt * 4), &full_bar[s]);
+                    bulk_load(st + ring.off_m + off * 4, a.m + si, uint32_t(cnt * 4), &full_bar[s]);
+                    bulk_load(st + ring.off_v + off * 4, a.v + si, uint32_t(cnt * 4), &full_bar[s]);
+                });
+            }
+        }
+        if (*abort_flag && lane == 0) {
+            // loads of the last tiles issued may still be landing: wait (bounded)
+            int dummy = 0;
+            volatile int *never = &dummy;
+            for (uint32_t i = 0; i < NS && i < k; ++i) {
+                const uint32_t kk = k - 1 - i;
+                mbar_wait(&full_bar[kk % NS], (kk / NS) & 1u, never);
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    // Group g takes the CTA's tiles k = g, g + GROUPS, ..., so one group's
+    // per-tile latency overlaps the other's.
+    const int ct = threadIdx.x - 32;
+    const uint32_t grp = uint32_t(ct) / kGroupThreads;
+    const uint32_t gt = uint32_t(ct) % kGroupThreads;
+    double acc = 0.0;
+    uint32_t bad = 0;
+    uint32_t k = grp;
+    for (uint64_t tile = blockIdx.x + uint64_t(grp) * gridDim.x; tile < n_tiles;
+         tile += uint64_t(GROUPS) * gridDim.x, k += GROUPS) {
+        const uint32_t s = k % NS;
+        bool failed = !mbar_wait(&full_bar[s], (k / NS) & 1u, abort_flag);
+        if (!failed && stage_tile[s] != tile) {  // self-check of the ring protocol
+            failed = true;
+            *abort_flag = 1;
+            atomicExch(&g_wait_error, 2);
+        }
+        const uint64_t jb = a.j0 + tile * T;
+        const uint32_t n = uint32_t(min(jb + T, a.j1) - jb);
+        const unsigned char *st = smem + size_t(s) * ring.stage_bytes;
+        if (!failed) {
+            const uint32_t nv = n >> 3;
+            for (uint32_t vv = gt; vv < nv; vv += kGroupThreads) {
+                const unsigned char *gp = st + size_t(vv) * 16;
+                float sum[8];
+                zero_dev::unpack8(lds128(gp), sum);
+#pragma unroll 4
+                for (uint32_t r = 1; r < a.nd; ++r) zero_dev::add8(sum, lds128(gp + size_t(r) * T * 2));
+                const float4 *wp = reinterpret_cast<const float4 *>(st + ring.off_w + size_t(vv) * 32);
+                const float4 *mp = reinterpret_cast<const float4 *>(st + ring.off_m + size_t(vv) * 32);
+                const float4 *vp = reinterpret_cast<const float4 *>(st + ring.off_v + size_t(vv) * 32);
+                const float4 w0 = wp[0], w1 = wp[1], m0 = mp[0], m1 = mp[1], v0 = vp[0], v1 = vp[1];
+                if (a.ws_mode) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        acc += double(sum[e]) * double(sum[e]);
+                        bad += zero_dev::not_finite(sum[e]);
+                    }
+                }
+                const uint64_t j = jb + uint64_t(vv) * 8;
+                const uint64_t o = OWNER_MAP ? j / a.shard : 0;
+                const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
+                const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
+                if (a.red) {
+                    __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(sum[0], sum[1], sum[2], sum[3]));
+                    __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(sum[4], sum[5], sum[6], sum[7]));
+                }
+                float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+                float vq[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) zero_dev::adam1(sum[e], a.c, wv[e], mv[e], vq[e]);
+                __stcs(reinterpret_cast<float4 *>(a.w + si), make_float4(wv[0], wv[1], wv[2], wv[3]));
+                __stcs(reinterpret_cast<float4 *>(a.w + si + 4), make_float4(wv[4], wv[5], wv[6], wv[7]));
+                __stcs(reinterpret_cast<float4 *>(a.m + si), make_float4(mv[0], mv[1], mv[2], mv[3]));
+                __stcs(reinterpret_cast<float4 *>(a.m + si + 4), make_float4(mv[4], mv[5], mv[6], mv[7]));
+                __stcs(reinterpret_cast<float4 *>(a.v + si), make_float4(vq[0], vq[1], vq[2], vq[3]));
+                __stcs(reinterpret_cast<float4 *>(a.v + si + 4), make_float4(vq[4], vq[5], vq[6], vq[7]));
+                uint4 pk;
+                pk.x = zero_dev::pack_bf16x2(wv[0], wv[1]);
+                pk.y = zero_dev::pack_bf16x2(wv[2], wv[3]);
+                pk.z = zero_dev::pack_bf16x2(wv[4], wv[5]);
+                pk.w = zero_dev::pack_bf16x2(wv[6], wv[7]);
+                uint16_t *pp = a.params + pi;
+                for (uint32_t r = 0; r < a.n_prow; ++r)
+                    __stcs(reinterpret_cast<uint4 *>(pp + uint64_t(r) * a.param_stride), pk);
+            }
+        }
+        // the whole group has read the stage (or the CTA is giving up): same
+        // decision in all of its threads, then hand the stage back
+        if (barrier_or(1 + grp, kGroupThreads, failed || *abort_flag)) break;
+        if (gt == 0) mbar_arrive(&empty_bar[s]);
+    }
+
+    if (a.ws_mode) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            acc += __shfl_down_sync(0xffffffffu, acc, off);
+            bad += __shfl_down_sync(0xffffffffu, bad, off);
+        }
+        if (lane == 0) {
+            s_norm[warp - 1] = acc;
+            s_bad[warp - 1] = bad;
+        }
+        barrier_or(1 + GROUPS, kConsumers, false);
+        if (ct == 0) {
+            double t = 0.0;
+            uint32_t b = 0;
+            for (int i = 0; i < kConsumerWarps; ++i) {
+                t += s_norm[i];
+                b += s_bad[i];
+            }
+            a.ws_norm[blockIdx.x] += t;
+            a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
+        }
+    }
+}
+
+}  // namespace zero_tma
