@@ -164,6 +164,23 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+# -------------------------------------------------------- multi-rank timing
+def max_over_ranks(seconds, dist, device):
+    """The slowest rank's device time (every rank gets the same value)."""
+    if dist is None:
+        return seconds
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, params_per_rank_step, steps, seconds):
+    """Whole-job Gparams/s: every rank updates its own replica of the
+    workload, so the job processes world x params per step."""
+    return world * params_per_rank_step * steps / seconds / 1e9
+
+
 # ----------------------------------------------------------------- workload
 class Workload:
     """Device buffers of one configuration, built from the seeded generators."""
@@ -371,10 +388,7 @@ def run_ours(args, cfg, rank, world, dist):
                 continue
             k1_time += events[k][b].elapsed_time(events[k][b + 1]) / 1e3
             k1_elems += wl.bucket_elems(b)
-    if dist is not None:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, dist, dev)
 
     # end to end through the public API: gradients from pinned host memory
     # every step, the step, the norm and overflow flag read back every step
@@ -406,11 +420,8 @@ def _e2e(args, wl, stream, dev, world, dist, t_first):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_t = e0.elapsed_time(e1) / 1e3
-    if dist is not None:
-        t = torch.tensor([e2e_t], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    return {"value": world * wl.params_per_step * e2e_steps / e2e_t / 1e9, "unit": UNIT,
+    e2e_t = max_over_ranks(e2e_t, dist, dev)
+    return {"value": job_value(world, wl.params_per_step, e2e_steps, e2e_t), "unit": UNIT,
             "h2d_bytes_per_step": Gh.numel() * Gh.element_size(),
             "d2h_bytes_per_step": 8 + 4, "steps": e2e_steps}
 
@@ -430,7 +441,7 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
             "algorithmic_bytes_per_launch": k1_bytes / n_launch,
             "avg_launch_ms": k1_time / n_launch * 1e3}
     step_bytes = wl.step_bytes + wl.gather_bytes
-    value = world * wl.params_per_step * args.steps / elapsed / 1e9
+    value = job_value(world, wl.params_per_step, args.steps, elapsed)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,

@@ -465,3 +465,30 @@ def test_oracle_never_imports_the_product():
             with open(os.path.join(here, name), encoding="utf-8") as f:
                 src = f.read()
             assert not re.search(r"zero_partitioned_optimizer_step_b200|libzero", src), name
+
+
+@pytest.mark.parametrize("stage,owner", [(2, None), (3, None), (2, 3)])
+def test_hbm_bytes_equal_bytes_of_buffers_the_step_touches(stage, owner):
+    """The accounting equals the sizes of the arrays one oracle step reads
+    (gradients, w, m, v) and writes (w, m, v, parameters, reduced gradient)."""
+    rng = np.random.default_rng(10)
+    units = [3000, 5000] if stage == 3 else None
+    pl = P.make_plan(8000, 8, stage, 2048, align=8, unit_elems=units)
+    G = rand_bf16(rng, (8, pl.psi_pad), 1e-3)
+    if owner is None:
+        w = np.zeros(8 * pl.S, np.float32)
+        m, v, red = w.copy(), w.copy(), w.copy()
+        params = (np.zeros(8 * pl.S, np.uint16) if stage == 3
+                  else np.zeros((8, pl.psi_pad), np.uint16))
+        ST.step_partitioned(pl, G, w, m, v, params, ADAM, 1, reduced=red)
+        reads = G.nbytes + w.nbytes + m.nbytes + v.nbytes
+    else:
+        Go = G[:, ST.owner_columns(pl, owner)]
+        w = np.zeros(pl.S, np.float32)
+        m, v = w.copy(), w.copy()
+        params, red, _, _ = ST.step_owner_view(pl, owner, Go, w, m, v, ADAM, 1, want_reduced=True)
+        reads = Go.nbytes + w.nbytes + m.nbytes + v.nbytes
+    writes = w.nbytes + m.nbytes + v.nbytes + params.nbytes
+    view = owner is not None
+    assert P.hbm_step_bytes(pl, owner_view=view) == reads + writes
+    assert P.hbm_step_bytes(pl, owner_view=view, with_reduced=True) == reads + writes + red.nbytes
