@@ -432,9 +432,10 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
     k1_bytes = per_elem * k1_elems
     achieved = k1_bytes / k1_time / 1e9
     n_launch = args.steps * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
-    tr = k1_traffic_per_elem() if (args.config == "c2" and args.psi is None) else None
-    roof = {"kernel": "k_step_tma (fused reduce-scatter + Adam + all-gather, one bucket; "
-                      "bulk-copy ring)",
+    tr = (k1_traffic_per_elem() if (args.config == "c2" and args.psi is None
+                                    and wl.Z.zero_step_kernel(wl.lp, wl.owner) == "k_step_tma") else None)
+    kname = wl.Z.zero_step_kernel(wl.lp, wl.owner)
+    roof = {"kernel": kname + " (fused reduce-scatter + Adam + all-gather, one bucket)",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
             "traffic": None if tr is None else tr * k1_elems / n_launch,

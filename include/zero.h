@@ -288,6 +288,15 @@ zero_status_t zero_bytes_moved(const zero_plan_t *plan, zero_bytes_kind_t kind,
  * steps, not inside a captured graph. */
 zero_status_t zero_stream_status(void *stream);
 
+#define ZERO_KERNEL_BULK_COPY 1u    /* k_step_tma: bulk-copy (TMA) shared-memory ring */
+#define ZERO_KERNEL_VECTOR_LOAD 2u  /* k_step_vec8: 16-byte vector loads */
+
+/* Which kernel zero_step() uses for the aligned bucket bodies of `plan` on
+ * the current CUDA device (owner_view as in zero_bufs_t), written to *kind.
+ * Queries the device once.  ZERO_EINVAL: NULL argument or owner_view out of
+ * range.  ZERO_ECUDA: the device query failed. */
+zero_status_t zero_step_kernel(const zero_plan_t *plan, int32_t owner_view, uint32_t *kind);
+
 /* Static text of a status code. */
 const char *zero_status_str(zero_status_t status);
 

@@ -100,6 +100,8 @@ def lib():
         L.zero_release_layer.argtypes = [vp, ctypes.c_uint32]
         L.zero_bytes_moved.restype = st
         L.zero_bytes_moved.argtypes = [vp, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(u64)]
+        L.zero_step_kernel.restype = st
+        L.zero_step_kernel.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)]
         L.zero_stream_status.restype = st
         L.zero_stream_status.argtypes = [vp]
         L.zero_status_str.restype = ctypes.c_char_p
@@ -311,6 +313,18 @@ def zero_gather_layer(plan, unit, owner_params, full_layer, stream=None):
                                    _ptr(owner_params, torch.bfloat16, "owner_params"),
                                    _ptr(full_layer, torch.bfloat16, "full_layer"),
                                    _stream(stream)))
+
+
+ZERO_KERNEL_BULK_COPY = 1
+ZERO_KERNEL_VECTOR_LOAD = 2
+
+
+def zero_step_kernel(plan, owner_view=-1):
+    """Name of the kernel zero_step uses for aligned bucket bodies on the
+    current device: 'k_step_tma' (bulk-copy ring) or 'k_step_vec8'."""
+    out = ctypes.c_uint32()
+    _check(lib().zero_step_kernel(plan.handle, int(owner_view), ctypes.byref(out)))
+    return "k_step_tma" if out.value == ZERO_KERNEL_BULK_COPY else "k_step_vec8"
 
 
 def zero_stream_status(stream=None):

@@ -245,7 +245,8 @@ __global__ void __launch_bounds__(kThreads) k_finalize(const double *ws_norm, co
 }
 
 // K2: full_layer[o*s_u + i] = owner_params[o*S + off_u + i] for the first
-// len_u elements; `cpo` CTAs per owner, owners in rank order.
+// len_u elements; `cpo` CTAs per owner, owners in rank order.  Each thread
+// keeps four 16-byte loads in flight before it stores them.
 __global__ void __launch_bounds__(kThreads) k_gather(const uint16_t *src, uint64_t S, uint64_t off_u,
                                                     uint64_t s_u, uint64_t len, uint16_t *dst,
                                                     uint32_t nd, uint32_t cpo, int vec_ok) {
@@ -260,13 +261,34 @@ __global__ void __launch_bounds__(kThreads) k_gather(const uint16_t *src, uint64
     const uint64_t nv = vec_ok ? (n >> 3) : 0;
     const uint4 *s4 = reinterpret_cast<const uint4 *>(s);
     uint4 *d4 = reinterpret_cast<uint4 *>(d);
-    for (uint64_t i = uint64_t(c) * kThreads + threadIdx.x; i < nv; i += stride) __stcs(d4 + i, __ldcs(s4 + i));
-    for (uint64_t i = (nv << 3) + uint64_t(c) * kThreads + threadIdx.x; i < n; i += stride) d[i] = s[i];
+    uint64_t i = uint64_t(c) * kThreads + threadIdx.x;
+    for (; i + 3 * stride < nv; i += 4 * stride) {
+        const uint4 x0 = __ldcs(s4 + i), x1 = __ldcs(s4 + i + stride);
+        const uint4 x2 = __ldcs(s4 + i + 2 * stride), x3 = __ldcs(s4 + i + 3 * stride);
+        __stcs(d4 + i, x0);
+        __stcs(d4 + i + stride, x1);
+        __stcs(d4 + i + 2 * stride, x2);
+        __stcs(d4 + i + 3 * stride, x3);
+    }
+    for (; i < nv; i += stride) __stcs(d4 + i, __ldcs(s4 + i));
+    for (uint64_t q = (nv << 3) + uint64_t(c) * kThreads + threadIdx.x; q < n; q += stride) d[q] = s[q];
 }
 
 // ----------------------------------------------------------------- host side
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The bulk-copy kernel instantiations: owner map x consumer groups x vector width.
+using TmaKernel = void (*)(const StepArgs, const zero_tma::Ring);
+
+template <bool OM>
+TmaKernel tma_kernel(uint32_t groups, uint32_t vw) {
+    if (groups == 2)
+        return vw == 2 ? zero_tma::k_step_tma<OM, 2, 2>
+                       : (vw == 4 ? zero_tma::k_step_tma<OM, 2, 4> : zero_tma::k_step_tma<OM, 2, 8>);
+    return vw == 2 ? zero_tma::k_step_tma<OM, 1, 2>
+                   : (vw == 4 ? zero_tma::k_step_tma<OM, 1, 4> : zero_tma::k_step_tma<OM, 1, 8>);
+}
 
 // Launch shapes of the step kernels on one device, computed once per device:
 // the persistent grid of the vector kernel (SM count x resident CTAs, capped
@@ -297,20 +319,19 @@ zero_status_t device_shapes(DeviceShapes *out) {
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_vec8<false, kRB, kMinB>, kThreads, 0);
     cudaFuncAttributes fa{};
-    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, zero_tma::k_step_tma<true, 2>);
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
     DeviceShapes d;
     d.sms = uint32_t(std::max(1, sms));
     d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
     const int64_t budget = int64_t(optin) - int64_t(fa.sharedSizeBytes) - 256;
     d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
     if (d.tma_smem > 0) {
-        const void *fns[] = {reinterpret_cast<const void *>(zero_tma::k_step_tma<true, 1>),
-                             reinterpret_cast<const void *>(zero_tma::k_step_tma<false, 1>),
-                             reinterpret_cast<const void *>(zero_tma::k_step_tma<true, 2>),
-                             reinterpret_cast<const void *>(zero_tma::k_step_tma<false, 2>)};
-        for (const void *f : fns)
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
+        for (uint32_t g : {1u, 2u})
+            for (uint32_t vw : {2u, 4u, 8u})
+                for (TmaKernel f : {tma_kernel<true>(g, vw), tma_kernel<false>(g, vw)})
+                    if (e == cudaSuccess)
+                        e = cudaFuncSetAttribute(reinterpret_cast<const void *>(f),
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
     }
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("device query: ") + cudaGetErrorString(e));
     cache[dev] = d;
@@ -323,13 +344,19 @@ uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
 // Shared-memory ring of the bulk-copy kernel for Nd gradient rows.  Each
 // tile pays a fixed synchronisation latency, so tiles are large; two consumer
 // groups help where a tile is cheap to compute.  Shapes measured best on B200
-// at 64 MB buckets (5e8 params):
-//   Nd <= 4: 2 groups, 2048-element tiles, 4 stages
-//   Nd <= 8: 1 group, 2048, 3       Nd <= 16: 2 groups, 2048, 2
-//   Nd <= 32: 2 groups, 1024, 2     Nd <= 64: 1 group, 512, 3
-// Beyond 64 ranks (or when the shape does not fit) the 16-byte-load kernel is
-// used.  With two groups the stage count is even (each group owns half the
-// stages).  ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS override the
+// at 64 MB buckets (5e8 params), as (groups, tile, stages, elements/thread):
+//   Nd <= 4: (2, 2048, 4, 8)     Nd <= 8: (1, 2048, 3, 8)
+//   Nd <= 16: (1, 1024, 4, 4)    Nd <= 32: (1, 1024, 2, 8)
+//   Nd <= 64: (1, 512, 3, 4)
+// Read-heavy steps (parameters written once: stage 3 or one owner) do better
+// with larger bulk copies, i.e. larger tiles: Nd <= 16 takes (1, 2048, 2, 8)
+// (the stage-3 1.3B workload at Nd = 16).  Beyond 64 ranks the 16-byte-load
+// kernel is used, and also for read-heavy steps with more than 32 ranks: there
+// every gradient row of a 512-element tile is a 1 KB bulk copy, and the rate
+// at which an SM completes such copies caps the read bandwidth (0.64 of copy
+// bandwidth against 0.80 for the load kernel, one owner of 64 ranks).  With
+// two groups the stage count is even (each group owns half the stages).
+// ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS / ZERO_TMA_VW override the
 // shape (tuning; a tile must be a positive multiple of 256).
 zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t groups) {
     zero_tma::Ring q;
@@ -343,31 +370,38 @@ zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t group
     return q;
 }
 
-bool choose_ring(uint32_t nd, uint32_t budget, zero_tma::Ring *r) {
-    long force_t = 0, force_s = 0, force_g = 0;
+bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, zero_tma::Ring *r) {
+    long force_t = 0, force_s = 0, force_g = 0, force_v = 0;
     if (const char *e = std::getenv("ZERO_TMA_TILE")) force_t = std::strtol(e, nullptr, 10);
     if (const char *e = std::getenv("ZERO_TMA_STAGES")) force_s = std::strtol(e, nullptr, 10);
     if (const char *e = std::getenv("ZERO_TMA_GROUPS")) force_g = std::strtol(e, nullptr, 10);
-    uint32_t groups, stages;
+    if (const char *e = std::getenv("ZERO_TMA_VW")) force_v = std::strtol(e, nullptr, 10);
+    uint32_t groups, stages, vw;
     uint64_t tile;
     if (force_t >= 256 && force_t % 256 == 0 && force_t <= 16384) {
         tile = uint64_t(force_t);
         groups = force_g == 2 ? 2 : 1;
         stages = force_s >= 2 ? uint32_t(std::min<long>(force_s, zero_tma::kMaxStages)) : zero_tma::kMaxStages;
+        const uint64_t busy = tile * groups / zero_tma::kConsumers;  // keep a group's threads busy
+        vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
     } else if (nd <= 4) {
-        groups = 2, tile = 2048, stages = 4;
+        groups = 2, tile = 2048, stages = 4, vw = 8;
     } else if (nd <= 8) {
-        groups = 1, tile = 2048, stages = 3;
+        groups = 1, tile = 2048, stages = 3, vw = 8;
+    } else if (nd <= 16 && read_heavy) {
+        groups = 1, tile = 2048, stages = 2, vw = 8;
     } else if (nd <= 16) {
-        groups = 2, tile = 2048, stages = 2;
+        groups = 1, tile = 1024, stages = 4, vw = 4;
     } else if (nd <= 32) {
-        groups = 2, tile = 1024, stages = 2;
-    } else if (nd <= 64) {
-        groups = 1, tile = 512, stages = 3;
+        groups = 1, tile = 1024, stages = 2, vw = 8;
+    } else if (nd <= 64 && !read_heavy) {
+        groups = 1, tile = 512, stages = 3, vw = 4;
     } else {
         return false;
     }
+    if (force_v == 2 || force_v == 4 || force_v == 8) vw = uint32_t(force_v);
     zero_tma::Ring q = ring_for(nd, tile, 0, groups);
+    q.vw = vw;
     uint64_t ns = std::min<uint64_t>(budget / q.stage_bytes, stages);
     ns -= ns % groups;  // every stage belongs to one group
     if (ns < 2) return false;
@@ -430,14 +464,9 @@ struct Launcher {
                 const uint64_t tiles = (j1 - j0 + ring.tile - 1) / ring.tile;
                 const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
                 const size_t smem = size_t(ring.stages) * ring.stage_bytes;
-                if (owner_map && ring.groups == 2)
-                    zero_tma::k_step_tma<true, 2><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
-                else if (owner_map)
-                    zero_tma::k_step_tma<true, 1><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
-                else if (ring.groups == 2)
-                    zero_tma::k_step_tma<false, 2><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
-                else
-                    zero_tma::k_step_tma<false, 1><<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
+                TmaKernel f = owner_map ? tma_kernel<true>(ring.groups, ring.vw)
+                                        : tma_kernel<false>(ring.groups, ring.vw);
+                f<<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
             } else if (vec) {
                 if (owner_map)
                     k_step_vec8<true, kRB, kMinB><<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
@@ -530,7 +559,8 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     L.stream = static_cast<cudaStream_t>(stream_);
     L.want_ws = b->grad_norm_sq || b->overflow;
     const int choice = kernel_choice();
-    L.use_tma = choice != 1 && choose_ring(p->nd, shapes.tma_smem, &L.ring);
+    L.use_tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, &L.ring)
+                            : choice != 1 && choose_ring(p->nd, a.n_prow == 1, shapes.tma_smem, &L.ring);
     if (L.want_ws && first == 0) {
         // the step's first call zeroes the per-CTA norm slots
         cudaError_t e = cudaMemsetAsync(b->workspace, 0, zero_detail::kWorkspaceBytes, L.stream);
@@ -609,10 +639,9 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
     DeviceShapes shapes;
     zero_status_t st = device_shapes(&shapes);
     if (st != ZERO_OK) return st;
-    const uint32_t grid = shapes.grid_ldg;
     const uint64_t s_u = p->unit_shard[unit], off = p->unit_offset[unit], len = p->unit_len[unit];
     const int vec_ok = ((p->S | off | s_u) & 7u) == 0;
-    const uint32_t cpo = std::max<uint32_t>(1, grid / p->nd);
+    const uint32_t cpo = std::max<uint32_t>(1, (shapes.sms * 8) / p->nd);  // 8 CTAs/SM
     const uint64_t blocks = uint64_t(cpo) * p->nd;
     if (blocks > 0x7fffffffull) return set_error(ZERO_EINVAL, "zero_gather_layer: nd too large for one launch");
     k_gather<<<uint32_t(blocks), kThreads, 0, static_cast<cudaStream_t>(stream_)>>>(
@@ -644,5 +673,23 @@ ZERO_API zero_status_t zero_stream_status(void *stream) {
                                 : "zero_stream_status: a bounded wait in the bulk-copy step kernel gave up; the "
                                   "outputs of the steps since the last check are not valid");
     }
+    return ZERO_OK;
+}
+
+ZERO_API zero_status_t zero_step_kernel(const zero_plan_t *p, int32_t owner_view, uint32_t *kind) {
+    zero_detail::clear_error();
+    if (!p || !kind) return set_error(ZERO_EINVAL, "zero_step_kernel: NULL argument");
+    if (owner_view < -1 || owner_view >= int64_t(p->nd))
+        return set_error(ZERO_EINVAL, "zero_step_kernel: owner_view must be -1 or a rank in [0, nd)");
+    DeviceShapes shapes;
+    zero_status_t st = device_shapes(&shapes);
+    if (st != ZERO_OK) return st;
+    const bool replicas = owner_view < 0 && p->stage <= 2;
+    zero_tma::Ring ring{};
+    const int choice = kernel_choice();
+    const bool tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, &ring)
+                                 : choice != 1 && choose_ring(p->nd, !replicas || p->nd == 1,
+                                                              shapes.tma_smem, &ring);
+    *kind = tma ? ZERO_KERNEL_BULK_COPY : ZERO_KERNEL_VECTOR_LOAD;
     return ZERO_OK;
 }

@@ -46,8 +46,10 @@ constexpr int kMaxStages = 8;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Shared-memory ring chosen on the host.  A stage holds Nd gradient rows of
-// `tile` bf16 at offset 0, then w, m, v (fp32).
+// `tile` bf16 at offset 0, then w, m, v (fp32).  `vw` is the per-thread
+// vector width the kernel was instantiated with.
 struct Ring {
+    uint32_t vw;
     uint32_t tile;
     uint32_t stages;  // a multiple of groups
     uint32_t groups;  // consumer groups the kernel was instantiated with
@@ -163,7 +165,69 @@ __device__ __forceinline__ uint4 lds128(const unsigned char *p) {
     return *reinterpret_cast<const uint4 *>(p);
 }
 
-template <bool OWNER_MAP, int GROUPS>
+// Per-thread vector of VW consecutive elements (VW = 2, 4 or 8): bf16 rows
+// read from shared memory as 4/8/16 bytes, fp32 state as 8/16/32 bytes, and
+// streaming global stores of the same widths.  The host picks VW so that a
+// tile keeps every consumer thread of a group busy.
+template <int VW>
+__device__ __forceinline__ void lds_bf16(const unsigned char *p, float f[VW]) {
+    if constexpr (VW == 2) {
+        const uint32_t x = *reinterpret_cast<const uint32_t *>(p);
+        f[0] = zero_dev::bf16lo(x);
+        f[1] = zero_dev::bf16hi(x);
+    } else if constexpr (VW == 4) {
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        f[0] = zero_dev::bf16lo(x.x); f[1] = zero_dev::bf16hi(x.x);
+        f[2] = zero_dev::bf16lo(x.y); f[3] = zero_dev::bf16hi(x.y);
+    } else {
+        zero_dev::unpack8(*reinterpret_cast<const uint4 *>(p), f);
+    }
+}
+
+template <int VW>
+__device__ __forceinline__ void lds_f32(const unsigned char *p, float f[VW]) {
+    if constexpr (VW == 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        f[0] = x.x; f[1] = x.y;
+    } else {
+#pragma unroll
+        for (int h = 0; h < VW / 4; ++h) {
+            const float4 x = reinterpret_cast<const float4 *>(p)[h];
+            f[4 * h] = x.x; f[4 * h + 1] = x.y; f[4 * h + 2] = x.z; f[4 * h + 3] = x.w;
+        }
+    }
+}
+
+template <int VW>
+__device__ __forceinline__ void stg_f32(float *p, const float f[VW]) {
+    if constexpr (VW == 2) {
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(f[0], f[1]));
+    } else {
+#pragma unroll
+        for (int h = 0; h < VW / 4; ++h)
+            __stcs(reinterpret_cast<float4 *>(p) + h, make_float4(f[4 * h], f[4 * h + 1], f[4 * h + 2], f[4 * h + 3]));
+    }
+}
+
+// bf16(w) of VW elements to `rows` rows `stride` elements apart
+template <int VW>
+__device__ __forceinline__ void stg_bf16_rows(uint16_t *p, const float w[VW], uint32_t rows, uint64_t stride) {
+    uint32_t pk[VW / 2];
+#pragma unroll
+    for (int h = 0; h < VW / 2; ++h) pk[h] = zero_dev::pack_bf16x2(w[2 * h], w[2 * h + 1]);
+    for (uint32_t r = 0; r < rows; ++r) {
+        uint16_t *q = p + uint64_t(r) * stride;
+        if constexpr (VW == 2) {
+            __stcs(reinterpret_cast<unsigned int *>(q), pk[0]);
+        } else if constexpr (VW == 4) {
+            __stcs(reinterpret_cast<uint2 *>(q), make_uint2(pk[0], pk[1]));
+        } else {
+            __stcs(reinterpret_cast<uint4 *>(q), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        }
+    }
+}
+
+template <bool OWNER_MAP, int GROUPS, int VW>
 __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, const Ring ring) {
     constexpr uint32_t kGroupThreads = kConsumers / GROUPS;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -257,51 +321,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
         const uint32_t n = uint32_t(min(jb + T, a.j1) - jb);
         const unsigned char *st = smem + size_t(s) * ring.stage_bytes;
         if (!failed) {
-            const uint32_t nv = n >> 3;
+            const uint32_t nv = n / VW;
             for (uint32_t vv = gt; vv < nv; vv += kGroupThreads) {
-                const unsigned char *gp = st + size_t(vv) * 16;
-                float sum[8];
-                zero_dev::unpack8(lds128(gp), sum);
+                const unsigned char *gp = st + size_t(vv) * (2 * VW);
+                float sum[VW], f[VW];
+                lds_bf16<VW>(gp, sum);
 #pragma unroll 4
-                for (uint32_t r = 1; r < a.nd; ++r) zero_dev::add8(sum, lds128(gp + size_t(r) * T * 2));
-                const float4 *wp = reinterpret_cast<const float4 *>(st + ring.off_w + size_t(vv) * 32);
-                const float4 *mp = reinterpret_cast<const float4 *>(st + ring.off_m + size_t(vv) * 32);
-                const float4 *vp = reinterpret_cast<const float4 *>(st + ring.off_v + size_t(vv) * 32);
-                const float4 w0 = wp[0], w1 = wp[1], m0 = mp[0], m1 = mp[1], v0 = vp[0], v1 = vp[1];
+                for (uint32_t r = 1; r < a.nd; ++r) {
+                    lds_bf16<VW>(gp + size_t(r) * T * 2, f);
+#pragma unroll
+                    for (int e = 0; e < VW; ++e) sum[e] = __fadd_rn(sum[e], f[e]);
+                }
+                float wv[VW], mv[VW], vq[VW];
+                lds_f32<VW>(st + ring.off_w + size_t(vv) * (4 * VW), wv);
+                lds_f32<VW>(st + ring.off_m + size_t(vv) * (4 * VW), mv);
+                lds_f32<VW>(st + ring.off_v + size_t(vv) * (4 * VW), vq);
                 if (a.ws_mode) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
+                    for (int e = 0; e < VW; ++e) {
                         acc += double(sum[e]) * double(sum[e]);
                         bad += zero_dev::not_finite(sum[e]);
                     }
                 }
-                const uint64_t j = jb + uint64_t(vv) * 8;
+                const uint64_t j = jb + uint64_t(vv) * VW;
                 const uint64_t o = OWNER_MAP ? j / a.shard : 0;
                 const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
                 const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
-                if (a.red) {
-                    __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(sum[0], sum[1], sum[2], sum[3]));
-                    __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(sum[4], sum[5], sum[6], sum[7]));
-                }
-                float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-                float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-                float vq[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                if (a.red) stg_f32<VW>(a.red + si, sum);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) zero_dev::adam1(sum[e], a.c, wv[e], mv[e], vq[e]);
-                __stcs(reinterpret_cast<float4 *>(a.w + si), make_float4(wv[0], wv[1], wv[2], wv[3]));
-                __stcs(reinterpret_cast<float4 *>(a.w + si + 4), make_float4(wv[4], wv[5], wv[6], wv[7]));
-                __stcs(reinterpret_cast<float4 *>(a.m + si), make_float4(mv[0], mv[1], mv[2], mv[3]));
-                __stcs(reinterpret_cast<float4 *>(a.m + si + 4), make_float4(mv[4], mv[5], mv[6], mv[7]));
-                __stcs(reinterpret_cast<float4 *>(a.v + si), make_float4(vq[0], vq[1], vq[2], vq[3]));
-                __stcs(reinterpret_cast<float4 *>(a.v + si + 4), make_float4(vq[4], vq[5], vq[6], vq[7]));
-                uint4 pk;
-                pk.x = zero_dev::pack_bf16x2(wv[0], wv[1]);
-                pk.y = zero_dev::pack_bf16x2(wv[2], wv[3]);
-                pk.z = zero_dev::pack_bf16x2(wv[4], wv[5]);
-                pk.w = zero_dev::pack_bf16x2(wv[6], wv[7]);
-                uint16_t *pp = a.params + pi;
-                for (uint32_t r = 0; r < a.n_prow; ++r)
-                    __stcs(reinterpret_cast<uint4 *>(pp + uint64_t(r) * a.param_stride), pk);
+                for (int e = 0; e < VW; ++e) zero_dev::adam1(sum[e], a.c, wv[e], mv[e], vq[e]);
+                stg_f32<VW>(a.w + si, wv);
+                stg_f32<VW>(a.m + si, mv);
+                stg_f32<VW>(a.v + si, vq);
+                stg_bf16_rows<VW>(a.params + pi, wv, a.n_prow, a.param_stride);
             }
         }
         // the whole group has read the stage (or the CTA is giving up): same
