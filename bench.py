@@ -67,6 +67,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--psi", type=int, default=None,
                     help="override the parameter count (flat single-unit workloads only)")
+    ap.add_argument("--shard", type=int, default=None,
+                    help="one-owner workloads: owner shard size (psi = nd * shard)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="stage-3 layer-wise workload: number of transformer blocks")
     return ap.parse_args()
 
 
@@ -79,6 +83,20 @@ def get_cfg(args):
         cfg["psi"] = args.psi
         cfg["workload"] = "flat vector psi=%d, Nd=%d, stage %d, %d-element buckets" % (
             args.psi, cfg["nd"], cfg["stage"], cfg["bucket_elems"])
+    if args.shard is not None:
+        if cfg["owner_view"] < 0:
+            raise SystemExit("--shard applies to one-owner workloads only")
+        cfg["psi"] = cfg["nd"] * args.shard
+        cfg["workload"] = "one owner, shard %d, Nd=%d, %d-element buckets" % (
+            args.shard, cfg["nd"], cfg["bucket_elems"])
+    if args.layers is not None:
+        if cfg["units"] is None:
+            raise SystemExit("--layers applies to the stage-3 layer-wise workload only")
+        from zero_partitioned_optimizer_step_b200.configs import stage3_units
+        cfg["units"] = stage3_units(layers=args.layers)
+        cfg["psi"] = sum(cfg["units"])
+        cfg["workload"] = "stage 3 layer-wise, %d x hidden 2048 (psi=%d), Nd=%d" % (
+            args.layers, cfg["psi"], cfg["nd"])
     return cfg
 
 

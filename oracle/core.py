@@ -30,10 +30,10 @@ def lib():
         L.oracle_bf16_rne_array.restype = None
         L.oracle_bf16_rne_array.argtypes = [_p, _p, _u64]
         L.oracle_adam_scalars.restype = None
-        L.oracle_adam_scalars.argtypes = [_f64, _f64, _f64, _f64, _f64, _u64, _p]
+        L.oracle_adam_scalars.argtypes = [_f64, _f64, _f64, _f64, _f64, _f64, _u64, _p]
         L.oracle_update.restype = None
         L.oracle_update.argtypes = [_u64, _u32, _p, _u64, _p, _p, _p, _p, _p,
-                                    _f64, _f64, _f64, _f64, _f64, _u64, _p, _p]
+                                    _f64, _f64, _f64, _f64, _f64, _f64, _f32, _u64, _p, _p]
         L.oracle_reduce.restype = None
         L.oracle_reduce.argtypes = [_u64, _u32, _p, _u64, _p]
         _LIB = L
@@ -59,11 +59,12 @@ def bf16_to_f32(b):
 
 
 def adam_scalars(adam, t):
-    """The eight fp32 constants of step t: grad_scale, b1, b2, eps, 1-b1,
-    1-b2, lr/(1-b1^t), 1/sqrt(1-b2^t)."""
-    out = np.zeros(8, dtype=np.float32)
+    """The nine fp32 constants of step t: grad_scale, b1, b2, eps, 1-b1,
+    1-b2, lr/(1-b1^t), 1/sqrt(1-b2^t), 1-lr*weight_decay."""
+    out = np.zeros(9, dtype=np.float32)
     lib().oracle_adam_scalars(adam["lr"], adam["beta1"], adam["beta2"],
-                              adam["eps"], adam["grad_scale"], t, _ptr(out))
+                              adam["eps"], adam["grad_scale"],
+                              adam.get("weight_decay", 0.0), t, _ptr(out))
     return out
 
 
@@ -76,11 +77,13 @@ def reduce(grads):
     return out
 
 
-def update(grads, w, m, v, adam, t, want_params=True, want_reduced=False):
+def update(grads, w, m, v, adam, t, want_params=True, want_reduced=False,
+           clip_coef=1.0):
     """The elementwise core on contiguous columns.
 
     grads: uint16 [nd, n]; w, m, v: fp32 [n], updated IN PLACE.
-    adam: dict with lr, beta1, beta2, eps, grad_scale.
+    adam: dict with lr, beta1, beta2, eps, grad_scale and optional
+    weight_decay (AdamW; default 0).  clip_coef: fp32 global-norm factor.
     Returns (params uint16 [n] or None, reduced fp32 [n] or None,
              norm_sq float, nonfinite int).
     """
@@ -94,6 +97,7 @@ def update(grads, w, m, v, adam, t, want_params=True, want_reduced=False):
     bad = np.zeros(1, dtype=np.int64)
     lib().oracle_update(n, nd, _ptr(grads), n, _ptr(w), _ptr(m), _ptr(v),
                         _ptr(p), _ptr(red), adam["grad_scale"], adam["lr"],
-                        adam["beta1"], adam["beta2"], adam["eps"], t,
+                        adam["beta1"], adam["beta2"], adam["eps"],
+                        adam.get("weight_decay", 0.0), float(np.float32(clip_coef)), t,
                         _ptr(norm), _ptr(bad))
     return p, red, float(norm[0]), int(bad[0])

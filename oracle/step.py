@@ -46,7 +46,7 @@ def step_replicated(nd, grads, w, m, v, adam, t, want_reduced=False):
 
 
 def step_partitioned(pl: Plan, grads, master, m, v, params, adam, t,
-                     reduced=None):
+                     reduced=None, clip_coef=1.0):
     """Stages 1-3 over all Nd logical ranks.
 
     grads: uint16 [nd, psi_pad], logical order (zero in the padding).
@@ -70,7 +70,8 @@ def step_partitioned(pl: Plan, grads, master, m, v, params, adam, t,
             m_ = m[st:st + s]
             v_ = v[st:st + s]
             p, red, nn, bb = core.update(cols, w_, m_, v_, adam, t,
-                                         want_reduced=reduced is not None)
+                                         want_reduced=reduced is not None,
+                                         clip_coef=clip_coef)
             norm += nn
             bad += bb
             if reduced is not None:
@@ -83,7 +84,7 @@ def step_partitioned(pl: Plan, grads, master, m, v, params, adam, t,
 
 
 def step_owner_view(pl: Plan, owner, grads_owner, master, m, v, adam, t,
-                    want_reduced=False):
+                    want_reduced=False, clip_coef=1.0):
     """One owner's part of the step.
 
     grads_owner: uint16 [nd, S]: for every rank, its gradient on the columns
@@ -92,7 +93,7 @@ def step_owner_view(pl: Plan, owner, grads_owner, master, m, v, adam, t,
     Returns (params uint16 [S], reduced fp32 [S] or None, norm_sq, nonfinite).
     """
     p, red, nn, bb = core.update(grads_owner, master, m, v, adam, t,
-                                 want_reduced=want_reduced)
+                                 want_reduced=want_reduced, clip_coef=clip_coef)
     return p, red, nn, bb
 
 
@@ -139,3 +140,48 @@ def storage_to_logical(pl: Plan, x_storage):
             st = o * pl.S + pl.unit_offset[u]
             out[lo:lo + s] = x_storage[st:st + s]
     return out
+
+
+# ------------------------------------------------------------- guarded step
+# Not on the pages: the usual mixed-precision guards around an optimizer
+# step, as torch.nn.utils.clip_grad_norm_ defines the clip and as dynamic
+# loss scaling skips a step whose gradients overflowed.
+CLIP_EPS = 1e-6
+
+
+def guard_coef(norm_sq_gsum, grad_scale, max_norm):
+    """Global-norm clip factor of the gradient Adam sees, g = g_sum*s:
+    total = |s| * sqrt(sum g_sum^2) (double), c = max_norm / (total + 1e-6),
+    clamped to at most 1 and rounded once to fp32.  max_norm <= 0: no clip.
+    A non-finite norm leaves the gradient unscaled (c = 1): skip_nonfinite
+    is the guard for that case."""
+    if max_norm <= 0 or not np.isfinite(norm_sq_gsum):
+        return np.float32(1.0)
+    total = abs(grad_scale) * np.sqrt(norm_sq_gsum)
+    return np.float32(min(1.0, max_norm / (total + CLIP_EPS)))
+
+
+def step_guarded(pl: Plan, grads, master, m, v, params, adam, t, max_norm,
+                 skip_nonfinite, reduced):
+    """Two passes.  1: the rank-order reduction of every element into
+    `reduced` (owner storage), its sum of squares and non-finite count.
+    2: unless skip_nonfinite and some sum is not finite, the step of
+    step_partitioned with g = (g_sum*s)*c.  Returns (norm_sq, nonfinite,
+    coef, skipped)."""
+    norm = 0.0
+    bad = 0
+    for o in range(pl.nd):
+        for u in range(len(pl.unit_pad)):
+            s = pl.unit_shard[u]
+            lo = pl.unit_base[u] + o * s
+            st = o * pl.S + pl.unit_offset[u]
+            red = core.reduce(grads[:, lo:lo + s])
+            reduced[st:st + s] = red
+            r64 = red.astype(np.float64)
+            norm += float(np.dot(r64, r64))
+            bad += int((~np.isfinite(red)).sum())
+    if skip_nonfinite and bad:
+        return norm, bad, np.float32(1.0), True
+    coef = guard_coef(norm, adam["grad_scale"], max_norm)
+    step_partitioned(pl, grads, master, m, v, params, adam, t, clip_coef=coef)
+    return norm, bad, coef, False

@@ -24,7 +24,12 @@
  *     m = b1*m + (1-b1)*g ;  v = b2*v + ((1-b2)*g)*g
  *     w = w - (lr/(1-b1^t)) * ( m / (sqrt(v)/sqrt(1-b2^t) + eps) )
  *  where the division by sqrt(1-b2^t) is taken as a multiplication by the
- *  host-precomputed 1/sqrt(1-b2^t).  The hyperparameters come in double, as
+ *  host-precomputed 1/sqrt(1-b2^t).  Two optional extensions: decoupled
+ *  weight decay (AdamW, Loshchilov & Hutter), w is first multiplied by
+ *  (1 - lr*wd); and a global-norm clip coefficient c <= 1 applied to the
+ *  gradient, g = (g_sum*s)*c.  With wd = 0 and c = 1 both multiplications are
+ *  exact (by 1), so the plain Adam result is unchanged bit for bit.  The
+ *  hyperparameters come in double, as
  *  optimizer settings usually do; b1, b2, eps and the gradient scale are
  *  used rounded to float, and 1-b1, 1-b2 are formed in double before their
  *  own rounding.  The pages do not fix the summation order
@@ -71,10 +76,11 @@ void oracle_bf16_rne_array(const float *x, uint16_t *out, uint64_t n)
  * and rounded once to float:
  *   sc[0] grad_scale   sc[1] b1        sc[2] b2        sc[3] eps
  *   sc[4] 1-b1         sc[5] 1-b2      sc[6] lr/(1-b1^t)
- *   sc[7] 1/sqrt(1-b2^t)
+ *   sc[7] 1/sqrt(1-b2^t)               sc[8] 1-lr*wd (AdamW decay)
  * b1^t and b2^t are C99 pow() in double. */
 void oracle_adam_scalars(double lr, double beta1, double beta2, double eps,
-                         double grad_scale, uint64_t t, float sc[8])
+                         double grad_scale, double weight_decay, uint64_t t,
+                         float sc[9])
 {
     double bc1 = 1.0 - pow(beta1, (double)t);
     double bc2 = 1.0 - pow(beta2, (double)t);
@@ -86,6 +92,7 @@ void oracle_adam_scalars(double lr, double beta1, double beta2, double eps,
     sc[5] = (float)(1.0 - beta2);
     sc[6] = (float)(lr / bc1);
     sc[7] = (float)(1.0 / sqrt(bc2));
+    sc[8] = (float)(1.0 - lr * weight_decay);
 }
 
 /* The reduce step for one element: the fp32 sum of the Nd ranks' bf16
@@ -103,12 +110,14 @@ static float reduce_in_rank_order(const uint16_t *grads, uint64_t rank_stride,
 }
 
 /* One Adam update of one element, exactly in the order stated above. */
-static void adam_element(float g_sum, const float sc[8], float *w, float *m,
-                         float *v)
+static void adam_element(float g_sum, const float sc[9], float clip_coef,
+                         float *w, float *m, float *v)
 {
     const float grad_scale = sc[0], beta1 = sc[1], beta2 = sc[2], eps = sc[3];
     const float omb1 = sc[4], omb2 = sc[5], step = sc[6], ibc2 = sc[7];
-    float g = g_sum * grad_scale;
+    const float decay = sc[8];
+    float g_scaled = g_sum * grad_scale;
+    float g = g_scaled * clip_coef;
 
     float m_old = beta1 * (*m);
     float m_new_part = omb1 * g;
@@ -124,7 +133,8 @@ static void adam_element(float g_sum, const float sc[8], float *w, float *m,
     float denom = root_hat + eps;
     float ratio = m_new / denom;
     float delta = step * ratio;
-    float w_new = (*w) - delta;
+    float w_decayed = (*w) * decay;
+    float w_new = w_decayed - delta;
 
     *m = m_new;
     *v = v_new;
@@ -136,17 +146,19 @@ static void adam_element(float g_sum, const float sc[8], float *w, float *m,
  * out contiguously (element e of rank r's gradient at grads[r*rank_stride+e]),
  *   reduce in rank order -> optional reduced_out[e]
  *   -> norm_sq += (double)g_sum^2, nonfinite += !isfinite(g_sum)
- *   -> Adam on w[e], m[e], v[e] -> p_out[e] = bf16(w[e]).
+ *   -> Adam (with optional AdamW decay and clip coefficient) on w[e], m[e],
+ *   v[e] -> p_out[e] = bf16(w[e]).
  * reduced_out, p_out, norm_sq and nonfinite may be NULL.
  */
 void oracle_update(uint64_t n, uint32_t nd, const uint16_t *grads,
                    uint64_t rank_stride, float *w, float *m, float *v,
                    uint16_t *p_out, float *reduced_out, double grad_scale,
                    double lr, double beta1, double beta2, double eps,
-                   uint64_t t, double *norm_sq, int64_t *nonfinite)
+                   double weight_decay, float clip_coef, uint64_t t,
+                   double *norm_sq, int64_t *nonfinite)
 {
-    float sc[8];
-    oracle_adam_scalars(lr, beta1, beta2, eps, grad_scale, t, sc);
+    float sc[9];
+    oracle_adam_scalars(lr, beta1, beta2, eps, grad_scale, weight_decay, t, sc);
     double acc = 0.0;
     int64_t bad = 0;
     for (uint64_t e = 0; e < n; ++e) {
@@ -154,7 +166,7 @@ void oracle_update(uint64_t n, uint32_t nd, const uint16_t *grads,
         if (reduced_out) reduced_out[e] = g_sum;
         acc += (double)g_sum * (double)g_sum;
         if (!isfinite(g_sum)) ++bad;
-        adam_element(g_sum, sc, &w[e], &m[e], &v[e]);
+        adam_element(g_sum, sc, clip_coef, &w[e], &m[e], &v[e]);
         if (p_out) p_out[e] = oracle_bf16_rne(w[e]);
     }
     if (norm_sq) *norm_sq += acc;

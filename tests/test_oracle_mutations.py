@@ -18,8 +18,8 @@ MUTATIONS = {
     "no_bias_correction_1": ("sc[6] = (float)(lr / bc1);", "sc[6] = (float)lr;"),
     "no_bias_correction_2": ("sc[7] = (float)(1.0 / sqrt(bc2));", "sc[7] = 1.0f;"),
     "second_moment_missing_g": ("float v_new_part = v_g * g;", "float v_new_part = v_g;"),
-    "update_sign": ("float w_new = (*w) - delta;", "float w_new = (*w) + delta;"),
-    "grad_scale_dropped": ("float g = g_sum * grad_scale;", "float g = g_sum;"),
+    "update_sign": ("float w_new = w_decayed - delta;", "float w_new = w_decayed + delta;"),
+    "grad_scale_dropped": ("float g_scaled = g_sum * grad_scale;", "float g_scaled = g_sum;"),
     "sum_starts_at_zero": ("float s = bf16_bits_to_float(grads[e]);\n    for (uint32_t r = 1;",
                            "float s = 0.0f;\n    for (uint32_t r = 0;"),
     "sum_reverse_order": ("float x = bf16_bits_to_float(grads[(uint64_t)r * rank_stride + e]);",
@@ -27,10 +27,17 @@ MUTATIONS = {
     "bf16_truncates": ("uint32_t rounded = u + 0x7fffu + lsb;", "uint32_t rounded = u + 0u * lsb;"),
     "bf16_ties_away": ("uint32_t rounded = u + 0x7fffu + lsb;", "uint32_t rounded = u + 0x8000u + 0u * lsb;"),
     "beta1_for_v": ("float v_old = beta2 * (*v);", "float v_old = beta1 * (*v);"),
+    "decay_after_update": ("float w_decayed = (*w) * decay;", "float w_decayed = ((*w) - delta) * decay + delta;"),
+    "decay_ignores_lr": ("sc[8] = (float)(1.0 - lr * weight_decay);", "sc[8] = (float)(1.0 - weight_decay);"),
+    "clip_ignored": ("float g = g_scaled * clip_coef;", "float g = g_scaled;"),
 }
 
 NUMERIC_PINS = ("reduce or bf16 or adam or closed_form or constant or zero_gradient "
-                "or norm or partitioned or owner_view")
+                "or norm or partitioned or owner_view or clip or guarded or weight_decay")
+
+
+PIN_FILES = [os.path.join(ROOT, "tests", f) for f in ("test_oracle_pins.py",
+                                                     "test_oracle_guard_pins.py")]
 
 
 def _run_mutant(name, tmp):
@@ -45,8 +52,9 @@ def _run_mutant(name, tmp):
                     mutated, "-o", lib, "-lm"], check=True)
     env = dict(os.environ, ORACLE_LIB=lib)
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-k", NUMERIC_PINS],
-                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+                        *PIN_FILES, "-k", NUMERIC_PINS],
+                       env=env, cwd=os.path.join(ROOT, "tests"), capture_output=True, text=True,
+                       timeout=600)
     return r.returncode, r.stdout[-1500:]
 
 
