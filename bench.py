@@ -59,7 +59,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
-    ap.add_argument("--nd", type=int, default=64)
+    ap.add_argument("--nd", type=int, default=None,
+                    help="logical ranks (bucket sweep point: default 64; other workloads: "
+                         "override their Nd)")
     ap.add_argument("--bucket-mb", type=int, default=64)
     ap.add_argument("--sweep", default=None, help="write the c5 grid as JSON lines here")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -76,7 +78,13 @@ def parse_args():
 
 def get_cfg(args):
     from zero_partitioned_optimizer_step_b200.configs import CONFIGS, c5_config
-    cfg = c5_config(args.nd, args.bucket_mb) if args.config == "c5" else dict(CONFIGS[args.config])
+    if args.config == "c5":
+        cfg = c5_config(args.nd or 64, args.bucket_mb)
+    else:
+        cfg = dict(CONFIGS[args.config])
+        if args.nd is not None:
+            cfg["nd"] = args.nd
+            cfg["workload"] += " (Nd overridden to %d)" % args.nd
     if args.psi is not None:
         if cfg["units"] is not None or cfg["owner_view"] >= 0:
             raise SystemExit("--psi applies to flat all-ranks workloads only")

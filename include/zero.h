@@ -70,7 +70,7 @@
 extern "C" {
 #endif
 
-#define ZERO_ABI_VERSION 1
+#define ZERO_ABI_VERSION 2
 
 typedef enum zero_status {
     ZERO_OK = 0,
@@ -153,15 +153,19 @@ zero_status_t zero_plan_query(const zero_plan_t *plan, zero_query_t what,
 
 /* Adam hyperparameters (double, as optimizer settings usually are).  Per
  * element, with constants rounded once to fp32 (b1, b2, eps, grad_scale,
- * 1-b1, 1-b2, step = lr/(1-b1^t), ibc2 = 1/sqrt(1-b2^t), powers by pow()):
- *   g = g_sum*grad_scale;  m = b1*m + (1-b1)*g;  v = b2*v + ((1-b2)*g)*g;
- *   w = w - step * (m / (sqrt(v)*ibc2 + eps));  p = bf16_rne(w)
- * each operation a separate round-to-nearest fp32 operation (no FMA).
- * This is textbook Adam (bias-corrected, eps outside the root, no weight
- * decay); [CP] "为什么需要它" names the state, the pages give no formula. */
+ * 1-b1, 1-b2, step = lr/(1-b1^t), ibc2 = 1/sqrt(1-b2^t), decay = 1-lr*wd,
+ * powers by pow()):
+ *   g = (g_sum*grad_scale)*c;  m = b1*m + (1-b1)*g;  v = b2*v + ((1-b2)*g)*g;
+ *   w = w*decay - step * (m / (sqrt(v)*ibc2 + eps));  p = bf16_rne(w)
+ * each operation a separate round-to-nearest fp32 operation (no FMA); c is
+ * 1 except in zero_step_guarded().  This is textbook Adam (bias-corrected,
+ * eps outside the root) with optional decoupled weight decay (AdamW; wd = 0
+ * gives plain Adam bit for bit); [CP] "为什么需要它" names the state, the
+ * pages give no formula. */
 typedef struct zero_adam {
     double lr, beta1, beta2, eps;
     double grad_scale;     /* 1/Nd averages the summed gradient */
+    double weight_decay;   /* decoupled (AdamW); 0 = Adam */
 } zero_adam_t;
 
 /* Device buffers of one step (all device pointers, 16-byte aligned). */
@@ -223,7 +227,7 @@ zero_status_t zero_step_buckets(const zero_plan_t *plan,
  * its own pool up front, a plain C caller with no allocator of its own, code
  * that must not allocate while it runs).  The paper has no counterpart: this
  * is a packaging choice of this library.  The norm/overflow scratch lives in a
- * 49,152-byte static array in device memory owned by the library, present on
+ * 49,408-byte static array in device memory owned by the library, present on
  * every GPU that loads it until the process exits; bufs->workspace and
  * bufs->workspace_bytes are ignored, every other field is as for zero_step.
  * No cudaMalloc, cudaFree or other allocating call is made.  The first call on
@@ -237,6 +241,29 @@ zero_status_t zero_step_buckets(const zero_plan_t *plan,
  * failed. */
 zero_status_t zero_step_noalloc(const zero_plan_t *plan, const zero_bufs_t *bufs,
                                 const zero_adam_t *adam, uint64_t t, void *stream);
+
+/* Guards of zero_step_guarded(); the pages have no counterpart (these are
+ * the usual mixed-precision guards around an optimizer step). */
+typedef struct zero_guard {
+    double max_grad_norm;  /* > 0: clip the global norm of g = g_sum*grad_scale
+                              to this (c = min(1, max/(norm + 1e-6))); 0: off */
+    int32_t skip_nonfinite;/* 1: if any g_sum is inf or NaN, change nothing */
+} zero_guard_t;
+
+/* The step with global-norm clipping and/or skipping on non-finite
+ * gradients, in two passes: (1) every bucket's rank-order reduction into
+ * bufs->reduced_grad with the sum of squares and the non-finite count; a
+ * one-block kernel then forms norm = |grad_scale| * sqrt(sum g_sum^2) (double)
+ * and c (fp32; 1 if the norm is not finite); (2) unless skipped, Adam from
+ * the reduced gradients with g = (g_sum*grad_scale)*c.  reduced_grad,
+ * grad_norm_sq, overflow and workspace are required (the norm reported is
+ * sum g_sum^2).  A skipped step leaves master, m, v and params unchanged;
+ * *overflow tells the caller.  Moves 2Nd + 8 + 24 + params bytes per element
+ * (zero_bytes_moved(ZERO_BYTES_HBM_GUARDED_STEP)).  ZERO_EINVAL as zero_step,
+ * or a missing required buffer, or max_grad_norm < 0 or not finite. */
+zero_status_t zero_step_guarded(const zero_plan_t *plan, const zero_bufs_t *bufs,
+                                const zero_adam_t *adam, const zero_guard_t *guard,
+                                uint64_t t, void *stream);
 
 /* Stage 3: materialise unit `unit` -- copy the Nd owners' bf16 slices of it,
  * in rank order, into full_layer[0 .. len_u) (padding dropped) -- and mark
@@ -265,8 +292,9 @@ typedef enum zero_bytes_kind {
                                            3(Nd-1)S at stage 3 */
     ZERO_BYTES_COMM_PER_RANK = 1,       /* the same in bytes (bf16) */
     ZERO_BYTES_HBM_STEP = 2,            /* bytes zero_step moves in HBM */
-    ZERO_BYTES_HBM_GATHER_STEP = 3      /* bytes of the stage-3 gathers of one
+    ZERO_BYTES_HBM_GATHER_STEP = 3,     /* bytes of the stage-3 gathers of one
                                            step (2 per unit: 4 B/element) */
+    ZERO_BYTES_HBM_GUARDED_STEP = 4     /* bytes zero_step_guarded moves */
 } zero_bytes_kind_t;
 
 #define ZERO_BYTES_FLAG_OWNER_VIEW 1u    /* HBM_STEP of one owner's shard */

@@ -179,6 +179,16 @@ def hbm_step_bytes(pl: Plan, owner_view: bool = False,
     return n * per
 
 
+def hbm_guarded_step_bytes(pl: Plan, owner_view: bool = False) -> int:
+    """The guarded step in two passes: the reduction reads the Nd bf16 rows
+    and writes the fp32 sum; the update reads the sum and w, m, v and writes
+    w, m, v and the parameters."""
+    n = pl.S if owner_view else pl.psi_pad
+    per = (2 * pl.nd + 4) + (4 + 24)
+    per += 2 if (owner_view or pl.stage == 3) else 2 * pl.nd
+    return n * per
+
+
 def hbm_gather_bytes(pl: Plan, gathers_per_unit: int = 2) -> int:
     """Stage 3 materialisation: read 2 B and write 2 B per element of each
     unit, `gathers_per_unit` times per step (forward, then backward)."""

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_function():
     assert len(names) >= 11
     for n in names:
         assert hasattr(L, n), n
-    assert L.zero_abi_version() == 1
+    assert L.zero_abi_version() == 2
 
 
 def test_status_strings():
@@ -69,6 +69,9 @@ def check_against_oracle(psi, nd, stage, bucket, align, units, every_index=True)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_STEP, Z.ZERO_BYTES_FLAG_REDUCED) == \
         OP.hbm_step_bytes(op, with_reduced=True)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GATHER_STEP) == OP.hbm_gather_bytes(op)
+    assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GUARDED_STEP) == OP.hbm_guarded_step_bytes(op)
+    assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GUARDED_STEP, Z.ZERO_BYTES_FLAG_OWNER_VIEW) == \
+        OP.hbm_guarded_step_bytes(op, owner_view=True)
 
 
 def test_plan_bit_exact_to_oracle_bruteforce():

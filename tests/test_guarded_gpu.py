@@ -1,0 +1,86 @@
+"""GPU parity of AdamW (decoupled weight decay) in the fused step, and of the
+two-pass guarded step (global-norm clipping, skip on non-finite gradients),
+against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import zero_partitioned_optimizer_step_b200 as Z
+from zero_cases import Case, f32, u16
+
+pytestmark = pytest.mark.gpu
+
+ADAMW = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.1)
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    yield
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+@pytest.mark.parametrize("psi,nd,stage,units", [(65_536, 4, 2, None), (300_001, 16, 3, [100_000, 200_001]),
+                                                (200_000, 64, 2, None)])
+def test_adamw_fused_bit_exact(kernel, psi, nd, stage, units, monkeypatch):
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
+    c = Case(psi, nd, stage, 1 << 16, units=units, config_id=12, adam=ADAMW)
+    for t in (1, 2, 3):
+        diff = c.step_and_compare(t)
+        assert all(v == 0 for v in diff.values()), diff
+
+
+@pytest.mark.parametrize("psi,nd,stage,units,align", [
+    (500_000, 8, 2, None, 64), (300_001, 16, 3, [100_000, 3, 199_998], 64), (77_777, 5, 1, None, 1)])
+def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align):
+    """A guard that never triggers gives the fused step's bits."""
+    a = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
+    b = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
+    for t in (1, 2):
+        G = a.grads(t)
+        a.run_gpu(G, t)
+        (diff, coef, skipped) = b.guarded_step_and_compare(t, 1e9, True, G)
+        assert coef == 1.0 and not skipped and all(v == 0 for v in diff.values()), diff
+        for x, y in ((a.w, b.w), (a.m, b.m), (a.v, b.v), (a.red, b.red)):
+            assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+        assert torch.equal(a.params.view(torch.int16), b.params.view(torch.int16))
+
+
+@pytest.mark.parametrize("psi,nd,stage,units", [(500_000, 8, 2, None),
+                                                (300_001, 16, 3, [100_000, 3, 199_998])])
+def test_guarded_clipping(psi, nd, stage, units):
+    c = Case(psi, nd, stage, 1 << 15, units=units, sigma=1e-2, config_id=14, adam=ADAMW)
+    for t in (1, 2, 3):
+        diff, coef, skipped = c.guarded_step_and_compare(t, 0.05, True)
+        assert 0 < coef < 1 and not skipped
+
+
+def test_guarded_skip_and_no_skip_on_nan():
+    c = Case(200_000, 4, 2, 50_000, config_id=15, adam=ADAMW)
+    c.guarded_step_and_compare(1, 0.5, True)
+    w, m, v, p = f32(c.w).copy(), f32(c.m).copy(), f32(c.v).copy(), u16(c.params).copy()
+    G = c.grads(2)
+    G[2, 999] = float("nan")
+    diff, coef, skipped = c.guarded_step_and_compare(2, 0.5, True, G)
+    assert skipped and int(c.ovf.item()) == 1 and np.isnan(f32(c.red)[999])
+    assert np.array_equal(f32(c.w), w) and np.array_equal(f32(c.m), m)
+    assert np.array_equal(f32(c.v), v) and np.array_equal(u16(c.params), p)
+    # without skipping, the NaN propagates into that element only; the
+    # non-finite norm leaves the gradient unclipped
+    diff, coef, skipped = c.guarded_step_and_compare(3, 0.5, False, c.grads(3))
+    assert not skipped and coef == 1.0
+
+
+def test_guarded_requires_its_buffers():
+    c = Case(10_000, 4, 2, 4096, config_id=16, with_reduced=False)
+    with pytest.raises(Z.ZeroError) as e:
+        Z.zero_step_guarded(c.lp, c.grads(1), c.w, c.m, c.v, c.params, c.adam, 1,
+                            max_grad_norm=1.0, grad_norm_sq=c.norm, overflow=c.ovf, workspace=c.ws)
+    assert e.value.status == Z.ZERO_EINVAL
+    c = Case(10_000, 4, 2, 4096, config_id=16)
+    with pytest.raises(Z.ZeroError):
+        Z.zero_step_guarded(c.lp, c.grads(1), c.w, c.m, c.v, c.params, c.adam, 1,
+                            max_grad_norm=-1.0, reduced_grad=c.red, grad_norm_sq=c.norm,
+                            overflow=c.ovf, workspace=c.ws)

@@ -141,3 +141,17 @@ def test_guarded_step_clips_and_skips():
     for x, y in ((w, w2), (m, m2), (v, v2)):
         assert np.array_equal(x.view(np.uint32), y.view(np.uint32))
     assert np.array_equal(params, p2)
+
+
+@pytest.mark.parametrize("stage", [2, 3])
+def test_guarded_hbm_bytes_equal_buffers_the_two_passes_touch(stage):
+    """Pass 1 reads the gradients and writes the reduced sum; pass 2 reads
+    the sum and w, m, v and writes w, m, v and the parameters."""
+    units = [2000, 3000] if stage == 3 else None
+    pl, G, w = _guarded_case(stage, units)
+    red = np.zeros_like(w)
+    params = (np.zeros(pl.nd * pl.S, np.uint16) if stage == 3
+              else np.zeros((pl.nd, pl.psi_pad), np.uint16))
+    pass1 = G.nbytes + red.nbytes
+    pass2 = red.nbytes + 2 * 3 * w.nbytes + params.nbytes
+    assert P.hbm_guarded_step_bytes(pl) == pass1 + pass2

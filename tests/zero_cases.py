@@ -130,6 +130,24 @@ class Case:
                     reduced_grad=self.red, grad_norm_sq=self.norm, overflow=self.ovf,
                     workspace=self.ws, owner_view=self.owner, **kw)
 
+    def run_gpu_guarded(self, G, t, max_norm, skip):
+        Z.zero_step_guarded(self.lp, G, self.w, self.m, self.v, self.params, self.adam, t,
+                            max_grad_norm=max_norm, skip_nonfinite=skip,
+                            reduced_grad=self.red, grad_norm_sq=self.norm, overflow=self.ovf,
+                            workspace=self.ws, owner_view=self.owner)
+
+    def guarded_step_and_compare(self, t, max_norm, skip, G=None):
+        """Two-pass guarded step against oracle.step.step_guarded."""
+        assert self.owner < 0 and self.red is not None and self.norm is not None
+        G = self.grads(t) if G is None else G
+        Gh = u16(G)
+        self.run_gpu_guarded(G, t, max_norm, skip)
+        norm, bad, coef, skipped = ST.step_guarded(self.op, Gh, self.hw, self.hm, self.hv,
+                                                   self.hparams, self.adam, t, max_norm, skip,
+                                                   self.hred)
+        Z.zero_stream_status()
+        return self.compare(norm, bad), coef, skipped
+
     def run_oracle(self, Gh, t):
         if self.owner >= 0:
             p, red, norm, bad = ST.step_owner_view(self.op, self.owner, Gh, self.hw, self.hm,

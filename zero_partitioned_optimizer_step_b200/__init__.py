@@ -31,7 +31,7 @@ ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ETIMEOUT = rang
 
 # accounting kinds (zero_bytes_kind_t) and flags
 (ZERO_BYTES_COMM_ELEMS_PER_RANK, ZERO_BYTES_COMM_PER_RANK, ZERO_BYTES_HBM_STEP,
- ZERO_BYTES_HBM_GATHER_STEP) = range(4)
+ ZERO_BYTES_HBM_GATHER_STEP, ZERO_BYTES_HBM_GUARDED_STEP) = range(5)
 ZERO_BYTES_FLAG_OWNER_VIEW = 1
 ZERO_BYTES_FLAG_REDUCED = 2
 
@@ -53,7 +53,11 @@ class _PlanDesc(ctypes.Structure):
 class _Adam(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double),
                 ("beta2", ctypes.c_double), ("eps", ctypes.c_double),
-                ("grad_scale", ctypes.c_double)]
+                ("grad_scale", ctypes.c_double), ("weight_decay", ctypes.c_double)]
+
+
+class _Guard(ctypes.Structure):
+    _fields_ = [("max_grad_norm", ctypes.c_double), ("skip_nonfinite", ctypes.c_int32)]
 
 
 class _Bufs(ctypes.Structure):
@@ -91,6 +95,9 @@ def lib():
         L.zero_step.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam), u64, vp]
         L.zero_step_noalloc.restype = st
         L.zero_step_noalloc.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam), u64, vp]
+        L.zero_step_guarded.restype = st
+        L.zero_step_guarded.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam),
+                                        ctypes.POINTER(_Guard), u64, vp]
         L.zero_step_buckets.restype = st
         L.zero_step_buckets.argtypes = [vp, ctypes.POINTER(_Bufs), ctypes.POINTER(_Adam),
                                         u64, u64, u64, vp]
@@ -278,6 +285,7 @@ def make_adam(adam):
     a.beta2 = float(adam["beta2"])
     a.eps = float(adam["eps"])
     a.grad_scale = float(adam["grad_scale"])
+    a.weight_decay = float(adam.get("weight_decay", 0.0))
     return a
 
 
@@ -297,6 +305,19 @@ def zero_step_noalloc(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t,
     b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
     _check(lib().zero_step_noalloc(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
                                    int(t), _stream(stream)))
+
+
+def zero_step_guarded(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t,
+                      max_grad_norm=0.0, skip_nonfinite=True, stream=None, **kw):
+    """The two-pass step with global-norm clipping and/or skipping on
+    non-finite gradients (reduced_grad, grad_norm_sq, overflow and workspace
+    are required keyword arguments)."""
+    b = make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, **kw)
+    g = _Guard()
+    g.max_grad_norm = float(max_grad_norm)
+    g.skip_nonfinite = 1 if skip_nonfinite else 0
+    _check(lib().zero_step_guarded(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
+                                   ctypes.byref(g), int(t), _stream(stream)))
 
 
 def zero_step_buckets(plan, grads, master, exp_avg, exp_avg_sq, params, adam, t,

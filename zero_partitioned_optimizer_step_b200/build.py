@@ -15,7 +15,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libzero.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("zero_plan.cpp", "zero_step.cu", "zero_noalloc.cu")]
-HEADERS = [os.path.join(CSRC, f) for f in ("zero_internal.h", "zero_device.cuh", "zero_tma.cuh")] + \
+HEADERS = [os.path.join(CSRC, f) for f in ("zero_internal.h", "zero_device.cuh", "zero_tma.cuh",
+                                             "zero_guard.cuh")] + \
     [os.path.join(ROOT, "include", "zero.h")]
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@ constexpr int kMinB = 2;  // CTAs per SM the vector kernel is sized for
 
 struct AdamConsts {
     float grad_scale, beta1, beta2, eps, omb1, omb2, step, ibc2;
+    float decay;  // 1 - lr * weight_decay (AdamW); 1 for Adam
 };
 
 // One launch: the unit-local element range [j0, j1) of one bucket.
@@ -64,17 +65,54 @@ __device__ __forceinline__ bool not_finite(float x) {
     return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
 }
 
-// Textbook Adam on one element, every operation rounded to nearest.
-__device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w, float &m,
-                                      float &v) {
-    const float g = __fmul_rn(g_sum, c.grad_scale);
+// Textbook Adam on one element with decoupled weight decay, every operation
+// rounded to nearest; g = (g_sum * grad_scale) * coef, where coef is the
+// global-norm clip factor of the guarded step (1 elsewhere; a multiplication
+// by 1, like the decay 1 of plain Adam, is exact).
+__device__ __forceinline__ void adam1c(float g_sum, float coef, const AdamConsts &c, float &w,
+                                       float &m, float &v) {
+    const float g = __fmul_rn(__fmul_rn(g_sum, c.grad_scale), coef);
     const float m_new = __fadd_rn(__fmul_rn(c.beta1, m), __fmul_rn(c.omb1, g));
     const float v_new = __fadd_rn(__fmul_rn(c.beta2, v), __fmul_rn(__fmul_rn(c.omb2, g), g));
     const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v_new), c.ibc2), c.eps);
     const float delta = __fmul_rn(c.step, __fdiv_rn(m_new, denom));
-    w = __fsub_rn(w, delta);
+    w = __fsub_rn(__fmul_rn(w, c.decay), delta);
     m = m_new;
     v = v_new;
+}
+
+__device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w, float &m,
+                                      float &v) {
+    adam1c(g_sum, 1.0f, c, w, m, v);
+}
+
+// Per-CTA partials of the gradient-norm / overflow reduction, added to slot
+// blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
+// so the reported norm is the same on every run of the same launch shapes.
+__device__ __forceinline__ void block_partials(double acc, uint32_t bad, const StepArgs &a) {
+    __shared__ double sd[kThreads / 32];
+    __shared__ uint32_t sb[kThreads / 32];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        acc += __shfl_down_sync(0xffffffffu, acc, off);
+        bad += __shfl_down_sync(0xffffffffu, bad, off);
+    }
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    if (lane == 0) {
+        sd[wid] = acc;
+        sb[wid] = bad;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        uint32_t b = 0;
+        for (int i = 0; i < kThreads / 32; ++i) {
+            t += sd[i];
+            b += sb[i];
+        }
+        a.ws_norm[blockIdx.x] += t;
+        a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
+    }
 }
 
 }  // namespace zero_dev

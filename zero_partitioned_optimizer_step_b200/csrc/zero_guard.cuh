@@ -1,0 +1,172 @@
+// Kernels of the guarded step (global-norm clipping, skip on non-finite
+// gradients), which needs the whole step's gradient norm before any update:
+//   k_reduce           pass 1: rank-order sum of the Nd bf16 rows into the
+//                      fp32 reduced gradient, per-CTA sums of squares and
+//                      non-finite counts (same arithmetic as the fused step);
+//   k_guard_finalize   one CTA: the fixed-order total, the clip coefficient
+//                      and the skip decision, written to the workspace;
+//   k_apply            pass 2: Adam from the reduced gradient, with
+//                      g = (g_sum * grad_scale) * coef, or nothing if skipped.
+// HBM-bound streams; 16-byte accesses on the vector path (VEC = 8), any
+// alignment on the scalar path (VEC = 1).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <cstdint>
+
+#include "zero_device.cuh"
+
+namespace zero_guarded {
+
+using zero_dev::AdamConsts;
+using zero_dev::StepArgs;
+using zero_dev::kThreads;
+
+struct GuardWord {
+    float coef;    // clip coefficient, <= 1
+    int32_t skip;  // 1: leave the state as it is
+};
+
+__device__ __forceinline__ uint64_t owner_of(const StepArgs &a, uint64_t j, bool owner_map) {
+    return owner_map ? j / a.shard : 0;
+}
+
+template <int VEC, bool OWNER_MAP>
+__global__ void __launch_bounds__(kThreads) k_reduce(const StepArgs a) {
+    const uint64_t n = (a.j1 - a.j0) / VEC;
+    const uint64_t stride = uint64_t(gridDim.x) * kThreads;
+    double acc = 0.0;
+    uint32_t bad = 0;
+    for (uint64_t vi = uint64_t(blockIdx.x) * kThreads + threadIdx.x; vi < n; vi += stride) {
+        const uint64_t j = a.j0 + vi * VEC;
+        const uint64_t o = owner_of(a, j, OWNER_MAP);
+        const uint64_t gi = uint64_t(a.g_base + int64_t(j));
+        const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
+        float s[VEC];
+        if constexpr (VEC == 8) {
+            const uint16_t *g = a.grads + gi;
+            uint4 x[4];
+            zero_dev::unpack8(__ldcs(reinterpret_cast<const uint4 *>(g)), s);
+            uint32_t r = 1;
+            for (; r + 4 <= a.nd; r += 4) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    x[k] = __ldcs(reinterpret_cast<const uint4 *>(g + uint64_t(r + k) * a.grad_stride));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) zero_dev::add8(s, x[k]);
+            }
+            for (; r < a.nd; ++r)
+                zero_dev::add8(s, __ldcs(reinterpret_cast<const uint4 *>(g + uint64_t(r) * a.grad_stride)));
+            __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(s[0], s[1], s[2], s[3]));
+            __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(s[4], s[5], s[6], s[7]));
+        } else {
+            s[0] = __uint_as_float(uint32_t(a.grads[gi]) << 16);
+            for (uint32_t r = 1; r < a.nd; ++r)
+                s[0] = __fadd_rn(s[0], __uint_as_float(uint32_t(a.grads[gi + uint64_t(r) * a.grad_stride]) << 16));
+            a.red[si] = s[0];
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            acc += double(s[e]) * double(s[e]);
+            bad += zero_dev::not_finite(s[e]);
+        }
+    }
+    zero_dev::block_partials(acc, bad, a);
+}
+
+// One CTA: sum the partials in a fixed order, report them, and decide.
+__global__ void __launch_bounds__(kThreads) k_guard_finalize(const double *ws_norm, const uint32_t *ws_bad,
+                                                            uint32_t slots, double *norm_out,
+                                                            int32_t *overflow_out, GuardWord *gw,
+                                                            double max_norm, double grad_scale,
+                                                            int skip_nonfinite) {
+    __shared__ double sd[kThreads];
+    __shared__ uint32_t sb[kThreads];
+    double t = 0.0;
+    uint32_t b = 0;
+    for (uint32_t i = threadIdx.x; i < slots; i += kThreads) {
+        t += ws_norm[i];
+        b |= ws_bad[i] != 0;
+    }
+    sd[threadIdx.x] = t;
+    sb[threadIdx.x] = b;
+    __syncthreads();
+    for (int s = kThreads / 2; s > 0; s >>= 1) {
+        if (threadIdx.x < s) {
+            sd[threadIdx.x] += sd[threadIdx.x + s];
+            sb[threadIdx.x] |= sb[threadIdx.x + s];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        const double norm_sq = sd[0];
+        *norm_out = norm_sq;
+        *overflow_out = sb[0] ? 1 : 0;
+        float coef = 1.0f;
+        if (max_norm > 0.0 && isfinite(norm_sq)) {
+            const double total = fabs(grad_scale) * sqrt(norm_sq);
+            coef = float(fmin(1.0, max_norm / (total + 1e-6)));
+        }
+        gw->coef = coef;
+        gw->skip = (skip_nonfinite && sb[0]) ? 1 : 0;
+    }
+}
+
+template <int VEC, bool OWNER_MAP>
+__global__ void __launch_bounds__(kThreads) k_apply(const StepArgs a, const GuardWord *gw) {
+    const GuardWord g = *gw;
+    if (g.skip) return;
+    const uint64_t n = (a.j1 - a.j0) / VEC;
+    const uint64_t stride = uint64_t(gridDim.x) * kThreads;
+    for (uint64_t vi = uint64_t(blockIdx.x) * kThreads + threadIdx.x; vi < n; vi += stride) {
+        const uint64_t j = a.j0 + vi * VEC;
+        const uint64_t o = owner_of(a, j, OWNER_MAP);
+        const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
+        const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
+        if constexpr (VEC == 8) {
+            float s[8], w[8], m[8], v[8];
+            const float4 *rp = reinterpret_cast<const float4 *>(a.red + si);
+            const float4 *wp = reinterpret_cast<const float4 *>(a.w + si);
+            const float4 *mp = reinterpret_cast<const float4 *>(a.m + si);
+            const float4 *vp = reinterpret_cast<const float4 *>(a.v + si);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float4 r4 = __ldcs(rp + h), w4 = __ldcs(wp + h), m4 = __ldcs(mp + h), v4 = __ldcs(vp + h);
+                s[4 * h] = r4.x; s[4 * h + 1] = r4.y; s[4 * h + 2] = r4.z; s[4 * h + 3] = r4.w;
+                w[4 * h] = w4.x; w[4 * h + 1] = w4.y; w[4 * h + 2] = w4.z; w[4 * h + 3] = w4.w;
+                m[4 * h] = m4.x; m[4 * h + 1] = m4.y; m[4 * h + 2] = m4.z; m[4 * h + 3] = m4.w;
+                v[4 * h] = v4.x; v[4 * h + 1] = v4.y; v[4 * h + 2] = v4.z; v[4 * h + 3] = v4.w;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) zero_dev::adam1c(s[e], g.coef, a.c, w[e], m[e], v[e]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                __stcs(reinterpret_cast<float4 *>(a.w + si) + h,
+                       make_float4(w[4 * h], w[4 * h + 1], w[4 * h + 2], w[4 * h + 3]));
+                __stcs(reinterpret_cast<float4 *>(a.m + si) + h,
+                       make_float4(m[4 * h], m[4 * h + 1], m[4 * h + 2], m[4 * h + 3]));
+                __stcs(reinterpret_cast<float4 *>(a.v + si) + h,
+                       make_float4(v[4 * h], v[4 * h + 1], v[4 * h + 2], v[4 * h + 3]));
+            }
+            uint4 pk;
+            pk.x = zero_dev::pack_bf16x2(w[0], w[1]);
+            pk.y = zero_dev::pack_bf16x2(w[2], w[3]);
+            pk.z = zero_dev::pack_bf16x2(w[4], w[5]);
+            pk.w = zero_dev::pack_bf16x2(w[6], w[7]);
+            for (uint32_t r = 0; r < a.n_prow; ++r)
+                __stcs(reinterpret_cast<uint4 *>(a.params + pi + uint64_t(r) * a.param_stride), pk);
+        } else {
+            float w = a.w[si], m = a.m[si], v = a.v[si];
+            zero_dev::adam1c(a.red[si], g.coef, a.c, w, m, v);
+            a.w[si] = w;
+            a.m[si] = m;
+            a.v[si] = v;
+            __nv_bfloat16 h = __float2bfloat16_rn(w);
+            const uint16_t bits = *reinterpret_cast<uint16_t *>(&h);
+            for (uint32_t r = 0; r < a.n_prow; ++r) a.params[pi + uint64_t(r) * a.param_stride] = bits;
+        }
+    }
+}
+
+}  // namespace zero_guarded

@@ -45,8 +45,10 @@ struct BucketRange {
 BucketRange bucket_range(const zero_plan_t &p, uint64_t b);
 
 // Workspace layout for the gradient-norm / overflow reduction: one fp64
-// partial and one u32 count per CTA slot, kMaxSlots slots.
+// partial and one u32 count per CTA slot, kMaxSlots slots, then 256 bytes
+// for the guarded step's decision (clip coefficient and skip flag).
 constexpr uint32_t kMaxSlots = 4096;
-constexpr uint64_t kWorkspaceBytes = uint64_t(kMaxSlots) * (8 + 4);
+constexpr uint64_t kGuardOffset = uint64_t(kMaxSlots) * (8 + 4);
+constexpr uint64_t kWorkspaceBytes = kGuardOffset + 256;
 
 }  // namespace zero_detail

@@ -22,7 +22,8 @@ using zero_detail::set_error;
 namespace {
 
 // Largest scratch the no-allocation entry point can use: one fp64 partial and
-// one u32 count per CTA slot of the step kernels (49,152 bytes).
+// one u32 count per CTA slot of the step kernels, plus the guarded step's
+// decision word (49,408 bytes).
 constexpr uint64_t kNoAllocScratchBytes = zero_detail::kWorkspaceBytes;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];

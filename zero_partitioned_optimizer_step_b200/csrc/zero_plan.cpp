@@ -238,6 +238,16 @@ ZERO_API zero_status_t zero_bytes_moved(const zero_plan_t *p, zero_bytes_kind_t 
             *out = n * per;
             return ZERO_OK;
         }
+        case ZERO_BYTES_HBM_GUARDED_STEP: {
+            // pass 1: Nd bf16 rows in, fp32 sum out; pass 2: fp32 sum and
+            // w, m, v in, w, m, v and the parameters out
+            const bool owner = flags & ZERO_BYTES_FLAG_OWNER_VIEW;
+            const uint64_t n = owner ? p->S : p->psi_pad;
+            uint64_t per = 2ull * p->nd + 4 + 4 + 24;
+            per += (owner || p->stage == 3) ? 2 : 2ull * p->nd;
+            *out = n * per;
+            return ZERO_OK;
+        }
         case ZERO_BYTES_HBM_GATHER_STEP: {
             uint64_t s = 0;
             for (uint64_t n : p->unit_len) s += 4 * n;

@@ -43,6 +43,7 @@
 #include <string>
 
 #include "zero_device.cuh"
+#include "zero_guard.cuh"
 #include "zero_tma.cuh"
 #include "zero_internal.h"
 
@@ -51,35 +52,6 @@ using zero_detail::set_error;
 namespace {
 
 using namespace zero_dev;
-
-// Per-CTA partials of the gradient-norm / overflow reduction, added to slot
-// blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
-// so the reported norm is the same on every run of the same launch shapes.
-__device__ __forceinline__ void block_partials(double acc, uint32_t bad, const StepArgs &a) {
-    __shared__ double sd[kThreads / 32];
-    __shared__ uint32_t sb[kThreads / 32];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        acc += __shfl_down_sync(0xffffffffu, acc, off);
-        bad += __shfl_down_sync(0xffffffffu, bad, off);
-    }
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (lane == 0) {
-        sd[wid] = acc;
-        sb[wid] = bad;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double t = 0.0;
-        uint32_t b = 0;
-        for (int i = 0; i < kThreads / 32; ++i) {
-            t += sd[i];
-            b += sb[i];
-        }
-        a.ws_norm[blockIdx.x] += t;
-        a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
-    }
-}
 
 // K1, vector path: 8 elements (16 B of bf16, 32 B of fp32) per thread and
 // iteration.  Preconditions (checked on the host): j0, j1, all bases, strides,
@@ -433,6 +405,7 @@ AdamConsts make_consts(const zero_adam_t &a, uint64_t t) {
     c.omb2 = float(1.0 - a.beta2);
     c.step = float(a.lr / bc1);
     c.ibc2 = float(1.0 / std::sqrt(bc2));
+    c.decay = float(1.0 - a.lr * a.weight_decay);
     return c;
 }
 
@@ -492,8 +465,9 @@ zero_status_t validate_step(const zero_plan_t *p, const zero_bufs_t *b, const ze
                             uint64_t t) {
     if (!p || !b || !adam) return set_error(ZERO_EINVAL, "zero_step: NULL argument");
     if (t == 0) return set_error(ZERO_EINVAL, "zero_step: t must be >= 1");
-    if (!(std::isfinite(adam->lr) && std::isfinite(adam->eps) && std::isfinite(adam->grad_scale)))
-        return set_error(ZERO_EINVAL, "zero_step: lr, eps and grad_scale must be finite");
+    if (!(std::isfinite(adam->lr) && std::isfinite(adam->eps) && std::isfinite(adam->grad_scale) &&
+          std::isfinite(adam->weight_decay)))
+        return set_error(ZERO_EINVAL, "zero_step: lr, eps, grad_scale and weight_decay must be finite");
     if (!(adam->beta1 >= 0.0 && adam->beta1 < 1.0 && adam->beta2 >= 0.0 && adam->beta2 < 1.0))
         return set_error(ZERO_EINVAL, "zero_step: beta1 and beta2 must be in [0, 1)");
     if (b->owner_view < -1 || b->owner_view >= int64_t(p->nd))
@@ -517,6 +491,82 @@ zero_status_t validate_step(const zero_plan_t *p, const zero_bufs_t *b, const ze
     return ZERO_OK;
 }
 
+// Launch arguments shared by every bucket of one call.
+StepArgs base_args(const zero_plan_t *p, const zero_bufs_t *b, const zero_adam_t *adam, uint64_t t) {
+    const bool replicas = b->owner_view < 0 && p->stage <= 2;
+    StepArgs a{};
+    a.grads = static_cast<const uint16_t *>(b->grads);
+    a.grad_stride = b->grad_stride;
+    a.w = b->master;
+    a.m = b->exp_avg;
+    a.v = b->exp_avg_sq;
+    a.red = b->reduced_grad;
+    a.params = static_cast<uint16_t *>(b->params);
+    a.param_stride = replicas ? b->param_stride : 0;
+    a.n_prow = replicas ? p->nd : 1;
+    a.nd = p->nd;
+    a.c = make_consts(*adam, t);
+    auto *ws = static_cast<unsigned char *>(b->workspace);
+    a.ws_norm = reinterpret_cast<double *>(ws);
+    a.ws_bad = reinterpret_cast<uint32_t *>(ws + 8ull * zero_detail::kMaxSlots);
+    return a;
+}
+
+// Arguments of bucket bk: its unit-local element range (the owner's part of
+// it in the one-owner view) and the offsets that map it to gradients, state
+// and parameters.  False if the bucket holds nothing for this view.
+bool bucket_args(const zero_plan_t *p, const zero_bufs_t *b, const StepArgs &a, uint64_t bk,
+                 StepArgs *out, bool *owner_map, bool *vec_ok) {
+    const bool owner = b->owner_view >= 0;
+    const bool replicas = !owner && p->stage <= 2;
+    const bool multi = p->unit_len.size() > 1;
+    const zero_detail::BucketRange br = zero_detail::bucket_range(*p, bk);
+    const uint32_t u = br.unit;
+    const uint64_t U = p->unit_base[u], s_u = p->unit_shard[u], O = p->unit_offset[u];
+    StepArgs x = a;
+    x.j0 = br.begin - U;
+    x.j1 = br.end - U;
+    *owner_map = false;
+    if (owner) {
+        const uint64_t lo = uint64_t(b->owner_view) * s_u, hi = lo + s_u;
+        x.j0 = std::max(x.j0, lo);
+        x.j1 = std::min(x.j1, hi);
+        if (x.j0 >= x.j1) return false;
+        x.g_base = x.s_base = x.p_base = int64_t(O) - int64_t(lo);
+        x.shard = x.jump = x.p_jump = 0;
+    } else {
+        x.g_base = int64_t(U);
+        x.s_base = int64_t(O);
+        if (multi) {
+            *owner_map = true;
+            x.shard = s_u;
+            x.jump = p->S - s_u;
+        }
+        x.p_base = replicas ? int64_t(U) : int64_t(O);
+        x.p_jump = replicas ? 0 : x.jump;
+    }
+    const bool strides_ok = (b->grad_stride & 7u) == 0 && (!replicas || (b->param_stride & 7u) == 0);
+    *vec_ok = strides_ok && mult8(x.g_base) && mult8(x.s_base) && mult8(x.p_base) &&
+              (!*owner_map || ((x.shard & 7u) == 0 && (x.jump & 7u) == 0));
+    *out = x;
+    return true;
+}
+
+// Calls f(j0, j1, vec) for the unaligned head, the 8-aligned body and the
+// unaligned tail of x's range (everything unaligned if !vec_ok).
+template <typename F>
+zero_status_t split_launch(const StepArgs &x, bool vec_ok, F f) {
+    if (x.j0 >= x.j1) return ZERO_OK;
+    if (!vec_ok) return f(x.j0, x.j1, false);
+    const uint64_t lo = (x.j0 + 7) & ~uint64_t(7), hi = x.j1 & ~uint64_t(7);
+    if (lo >= hi) return f(x.j0, x.j1, false);
+    zero_status_t s = ZERO_OK;
+    if (x.j0 < lo) s = f(x.j0, lo, false);
+    if (s == ZERO_OK) s = f(lo, hi, true);
+    if (s == ZERO_OK && hi < x.j1) s = f(hi, x.j1, false);
+    return s;
+}
+
 }  // namespace
 
 ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t *b,
@@ -534,25 +584,7 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     st = device_shapes(&shapes);
     if (st != ZERO_OK) return st;
 
-    const bool owner = b->owner_view >= 0;
-    const bool replicas = !owner && p->stage <= 2;
-    const bool multi = p->unit_len.size() > 1;
-
-    StepArgs a{};
-    a.grads = static_cast<const uint16_t *>(b->grads);
-    a.grad_stride = b->grad_stride;
-    a.w = b->master;
-    a.m = b->exp_avg;
-    a.v = b->exp_avg_sq;
-    a.red = b->reduced_grad;
-    a.params = static_cast<uint16_t *>(b->params);
-    a.param_stride = replicas ? b->param_stride : 0;
-    a.n_prow = replicas ? p->nd : 1;
-    a.nd = p->nd;
-    a.c = make_consts(*adam, t);
-    auto *ws = static_cast<unsigned char *>(b->workspace);
-    a.ws_norm = reinterpret_cast<double *>(ws);
-    a.ws_bad = reinterpret_cast<uint32_t *>(ws + 8ull * zero_detail::kMaxSlots);
+    const StepArgs a = base_args(p, b, adam, t);
 
     Launcher L;
     L.shapes = shapes;
@@ -568,35 +600,10 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
             return set_error(ZERO_ECUDA, std::string("zero_step workspace reset: ") + cudaGetErrorString(e));
     }
 
-    const bool strides_ok = (b->grad_stride & 7u) == 0 && (!replicas || (b->param_stride & 7u) == 0);
     for (uint64_t bk = first; bk < first + count; ++bk) {
-        const zero_detail::BucketRange br = zero_detail::bucket_range(*p, bk);
-        const uint32_t u = br.unit;
-        const uint64_t U = p->unit_base[u], s_u = p->unit_shard[u], O = p->unit_offset[u];
-        StepArgs x = a;
-        x.j0 = br.begin - U;
-        x.j1 = br.end - U;
-        bool owner_map = false;
-        if (owner) {
-            const uint64_t lo = uint64_t(b->owner_view) * s_u, hi = lo + s_u;
-            x.j0 = std::max(x.j0, lo);
-            x.j1 = std::min(x.j1, hi);
-            if (x.j0 >= x.j1) continue;
-            x.g_base = x.s_base = x.p_base = int64_t(O) - int64_t(lo);
-            x.shard = x.jump = x.p_jump = 0;
-        } else {
-            x.g_base = int64_t(U);
-            x.s_base = int64_t(O);
-            if (multi) {
-                owner_map = true;
-                x.shard = s_u;
-                x.jump = p->S - s_u;
-            }
-            x.p_base = replicas ? int64_t(U) : int64_t(O);
-            x.p_jump = replicas ? 0 : x.jump;
-        }
-        const bool vec_ok = strides_ok && mult8(x.g_base) && mult8(x.s_base) && mult8(x.p_base) &&
-                            (!owner_map || ((x.shard & 7u) == 0 && (x.jump & 7u) == 0));
+        StepArgs x;
+        bool owner_map, vec_ok;
+        if (!bucket_args(p, b, a, bk, &x, &owner_map, &vec_ok)) continue;
         st = L.run(x, owner_map, vec_ok);
         if (st != ZERO_OK) return st;
     }
@@ -691,5 +698,75 @@ ZERO_API zero_status_t zero_step_kernel(const zero_plan_t *p, int32_t owner_view
                                  : choice != 1 && choose_ring(p->nd, !replicas || p->nd == 1,
                                                               shapes.tma_smem, &ring);
     *kind = tma ? ZERO_KERNEL_BULK_COPY : ZERO_KERNEL_VECTOR_LOAD;
+    return ZERO_OK;
+}
+
+ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t *b, const zero_adam_t *adam,
+                                         const zero_guard_t *guard, uint64_t t, void *stream_) {
+    zero_detail::clear_error();
+    zero_status_t st = validate_step(p, b, adam, t);
+    if (st != ZERO_OK) return st;
+    if (!guard) return set_error(ZERO_EINVAL, "zero_step_guarded: NULL guard");
+    if (!(std::isfinite(guard->max_grad_norm) && guard->max_grad_norm >= 0.0))
+        return set_error(ZERO_EINVAL, "zero_step_guarded: max_grad_norm must be finite and >= 0");
+    if (!b->reduced_grad || !b->grad_norm_sq || !b->overflow || !b->workspace)
+        return set_error(ZERO_EINVAL,
+                         "zero_step_guarded: reduced_grad, grad_norm_sq, overflow and workspace are required");
+    cudaError_t pre = cudaPeekAtLastError();
+    if (pre != cudaSuccess)
+        return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_step_guarded: ") +
+                                         cudaGetErrorString(pre));
+    DeviceShapes shapes;
+    st = device_shapes(&shapes);
+    if (st != ZERO_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    StepArgs a = base_args(p, b, adam, t);
+    a.ws_mode = 1;
+    auto *gw = reinterpret_cast<zero_guarded::GuardWord *>(static_cast<unsigned char *>(b->workspace) +
+                                                         zero_detail::kGuardOffset);
+    cudaError_t e = cudaMemsetAsync(b->workspace, 0, zero_detail::kWorkspaceBytes, stream);
+    if (e != cudaSuccess)
+        return set_error(ZERO_ECUDA, std::string("zero_step_guarded workspace reset: ") + cudaGetErrorString(e));
+    const uint32_t grid = shapes.grid_ldg;
+    // pass 1: reductions, sums of squares, non-finite counts
+    for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
+        StepArgs x;
+        bool om, vec_ok;
+        if (!bucket_args(p, b, a, bk, &x, &om, &vec_ok)) continue;
+        st = split_launch(x, vec_ok, [&](uint64_t j0, uint64_t j1, bool vec) -> zero_status_t {
+            StepArgs y = x;
+            y.j0 = j0;
+            y.j1 = j1;
+            if (vec && om) zero_guarded::k_reduce<8, true><<<grid, kThreads, 0, stream>>>(y);
+            else if (vec) zero_guarded::k_reduce<8, false><<<grid, kThreads, 0, stream>>>(y);
+            else if (om) zero_guarded::k_reduce<1, true><<<grid, kThreads, 0, stream>>>(y);
+            else zero_guarded::k_reduce<1, false><<<grid, kThreads, 0, stream>>>(y);
+            return check_launch("zero_step_guarded reduce launch");
+        });
+        if (st != ZERO_OK) return st;
+    }
+    zero_guarded::k_guard_finalize<<<1, kThreads, 0, stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots,
+                                                             b->grad_norm_sq, b->overflow, gw,
+                                                             guard->max_grad_norm, adam->grad_scale,
+                                                             guard->skip_nonfinite ? 1 : 0);
+    st = check_launch("zero_step_guarded finalize launch");
+    if (st != ZERO_OK) return st;
+    // pass 2: Adam from the reduced gradients (no-op when the step is skipped)
+    for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
+        StepArgs x;
+        bool om, vec_ok;
+        if (!bucket_args(p, b, a, bk, &x, &om, &vec_ok)) continue;
+        st = split_launch(x, vec_ok, [&](uint64_t j0, uint64_t j1, bool vec) -> zero_status_t {
+            StepArgs y = x;
+            y.j0 = j0;
+            y.j1 = j1;
+            if (vec && om) zero_guarded::k_apply<8, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            else if (vec) zero_guarded::k_apply<8, false><<<grid, kThreads, 0, stream>>>(y, gw);
+            else if (om) zero_guarded::k_apply<1, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            else zero_guarded::k_apply<1, false><<<grid, kThreads, 0, stream>>>(y, gw);
+            return check_launch("zero_step_guarded apply launch");
+        });
+        if (st != ZERO_OK) return st;
+    }
     return ZERO_OK;
 }
