@@ -143,7 +143,16 @@ typedef enum zero_query {
     ZERO_Q_IS_LIVE = 22,        /* idx = u: 1 if unit u is live */
     ZERO_Q_MAX_LIVE = 23,
     ZERO_Q_ALIGN = 24,
-    ZERO_Q_BUCKET_ELEMS = 25
+    ZERO_Q_BUCKET_ELEMS = 25,
+    ZERO_Q_STATE_REPLICAS = 26, /* ranks holding each element's optimizer
+                                   state: Nd at stage 0, else 1 */
+    ZERO_Q_GRAD_REPLICAS = 27,  /* ... its reduced gradient: Nd at stages 0-1 */
+    ZERO_Q_PARAM_REPLICAS = 28, /* ... its parameter: Nd at stages 0-2 */
+    ZERO_Q_LOST_RANK_UNRECOVERABLE = 29 /* idx = rank r: parameters whose
+                                   optimizer state is lost with no other copy
+                                   if rank r is lost (its real, unpadded owned
+                                   elements when state is sharded; 0 at
+                                   stage 0) */
 } zero_query_t;
 
 /* Read one value of the plan into *out.  Host only.  ZERO_EINVAL: NULL
@@ -264,6 +273,20 @@ typedef struct zero_guard {
 zero_status_t zero_step_guarded(const zero_plan_t *plan, const zero_bufs_t *bufs,
                                 const zero_adam_t *adam, const zero_guard_t *guard,
                                 uint64_t t, void *stream);
+
+/* Reshard a checkpoint: copy one state array (fp32 master, m, v: elem_bytes
+ * 4; bf16 owner parameters: 2) from owner storage under plan `from`
+ * ([from.Nd * from.S]) to owner storage under plan `to` ([to.Nd * to.S]),
+ * element by element through the logical order; the destination's padding is
+ * written as zero.  The two plans must have the same unit lengths (the same
+ * model); Nd, alignment, stage and buckets may differ.  A checkpoint is then
+ * the owner-storage arrays plus t; resuming with another Nd is one call per
+ * array.  The concept page's "使用时应检查" list asks whether a checkpoint can
+ * be restored after the parallelism changes; this is that step.
+ * ZERO_EINVAL: NULL, elem_bytes not 2 or 4, different units, misaligned
+ * buffers.  ZERO_ECUDA: launch failure.  The buffers must not overlap. */
+zero_status_t zero_reshard(const zero_plan_t *from, const void *src, const zero_plan_t *to, void *dst,
+                           uint32_t elem_bytes, void *stream);
 
 /* Stage 3: materialise unit `unit` -- copy the Nd owners' bf16 slices of it,
  * in rank order, into full_layer[0 .. len_u) (padding dropped) -- and mark

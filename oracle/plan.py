@@ -207,3 +207,27 @@ def storage_index(pl: Plan, cols):
     owner = j // s
     off = np.asarray(pl.unit_offset, dtype=np.int64)[u] + (j - owner * s)
     return owner * pl.S + off
+
+
+# ------------------------------------------------------ replicas, rank loss
+def replicas(pl: Plan, what: str) -> int:
+    """Ranks that hold a copy of each element's state, gradient or parameter.
+    Concept page "ZeRO", table "三个阶段": ZeRO-1 shards the optimizer
+    states (parameters and gradients stay replicated on every rank), ZeRO-2
+    also the gradients, ZeRO-3 also the parameters; plain data parallelism
+    (stage 0) replicates everything."""
+    sharded_from = {"state": 1, "grad": 2, "param": 3}[what]
+    return 1 if pl.stage >= sharded_from else pl.nd
+
+
+def lost_rank_unrecoverable(pl: Plan, rank: int) -> int:
+    """Real (unpadded) parameters whose optimizer state has no other copy once
+    `rank` is lost: the ones it owns, unless the state is replicated."""
+    if replicas(pl, "state") > 1:
+        return 0
+    n = 0
+    for p in range(pl.psi_pad):
+        u, owner, _, j = locate(pl, p)
+        if owner == rank and j < pl.unit_len[u]:
+            n += 1
+    return n

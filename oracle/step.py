@@ -185,3 +185,16 @@ def step_guarded(pl: Plan, grads, master, m, v, params, adam, t, max_norm,
     coef = guard_coef(norm, adam["grad_scale"], max_norm)
     step_partitioned(pl, grads, master, m, v, params, adam, t, clip_coef=coef)
     return norm, bad, coef, False
+
+
+def reshard(pl_from: Plan, x, pl_to: Plan):
+    """A checkpointed owner-storage array under `pl_from`, laid out for
+    `pl_to` (same unit lengths): element (unit u, index j < len_u) keeps its
+    value; the new padding is zero."""
+    assert pl_from.unit_len == pl_to.unit_len
+    logical_a = storage_to_logical(pl_from, x)
+    logical_b = np.zeros(pl_to.psi_pad, dtype=x.dtype)
+    for u, n in enumerate(pl_to.unit_len):
+        a0, b0 = pl_from.unit_base[u], pl_to.unit_base[u]
+        logical_b[b0:b0 + n] = logical_a[a0:a0 + n]
+    return logical_to_storage(pl_to, logical_b)

@@ -69,6 +69,12 @@ def check_against_oracle(psi, nd, stage, bucket, align, units, every_index=True)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_STEP, Z.ZERO_BYTES_FLAG_REDUCED) == \
         OP.hbm_step_bytes(op, with_reduced=True)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GATHER_STEP) == OP.hbm_gather_bytes(op)
+    for q, what in ((Z.ZERO_Q_STATE_REPLICAS, "state"), (Z.ZERO_Q_GRAD_REPLICAS, "grad"),
+                    (Z.ZERO_Q_PARAM_REPLICAS, "param")):
+        assert lp.query(q) == OP.replicas(op, what)
+    if every_index:
+        for r in range(nd):
+            assert lp.query(Z.ZERO_Q_LOST_RANK_UNRECOVERABLE, r) == OP.lost_rank_unrecoverable(op, r)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GUARDED_STEP) == OP.hbm_guarded_step_bytes(op)
     assert Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_GUARDED_STEP, Z.ZERO_BYTES_FLAG_OWNER_VIEW) == \
         OP.hbm_guarded_step_bytes(op, owner_view=True)
@@ -206,3 +212,16 @@ def test_product_never_imports_the_oracle():
             if f.endswith((".py", ".cu", ".cpp", ".h")):
                 src = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert not re.search(r"\boracle\b\s*(import|\.)|from\s+oracle|liboracle", src), f
+
+
+def test_reshard_argument_checks_on_host():
+    L = Z.lib()
+    a = Z.zero_plan(1000, 4, 2, 100, unit_elems=[400, 600])
+    b = Z.zero_plan(1000, 3, 3, 100, unit_elems=[400, 600])
+    c = Z.zero_plan(1000, 3, 3, 100, unit_elems=[500, 500])
+    ok = ctypes.c_void_p(4096)
+    assert L.zero_reshard(a.handle, ok, c.handle, ctypes.c_void_p(8192), 4, None) == Z.ZERO_EINVAL
+    assert L.zero_reshard(a.handle, ok, b.handle, ctypes.c_void_p(8192), 8, None) == Z.ZERO_EINVAL
+    assert L.zero_reshard(a.handle, None, b.handle, ctypes.c_void_p(8192), 4, None) == Z.ZERO_EINVAL
+    assert L.zero_reshard(a.handle, ctypes.c_void_p(4098), b.handle, ctypes.c_void_p(8192), 4,
+                          None) == Z.ZERO_EINVAL

@@ -492,3 +492,47 @@ def test_hbm_bytes_equal_bytes_of_buffers_the_step_touches(stage, owner):
     view = owner is not None
     assert P.hbm_step_bytes(pl, owner_view=view) == reads + writes
     assert P.hbm_step_bytes(pl, owner_view=view, with_reduced=True) == reads + writes + red.nbytes
+
+
+def test_replicas_follow_the_stage_table():
+    rows = read_golden("stage_table.txt")
+    for st, state, grad, param in rows:
+        pl = P.make_plan(1000, 8, int(st), 100)
+        for what, mark in (("state", state), ("grad", grad), ("param", param)):
+            assert P.replicas(pl, what) == (1 if mark == "S" else 8), (st, what)
+    # the memory model agrees: a replicated state costs its full size per rank
+    for st, state, grad, param in rows:
+        pl = P.make_plan(64_000, 8, int(st), 100, align=1)
+        want = sum(b * (pl.psi if mark == "R" else pl.psi // 8)
+                   for b, mark in ((12, state), (2, grad), (2, param)))
+        assert P.memory_bytes_per_rank_padded(pl, int(st)) == want
+
+
+def test_lost_rank_counts_owned_real_elements():
+    pl = P.make_plan(100, 3, 2, 10, align=4, unit_elems=[37, 63])
+    counts = [P.lost_rank_unrecoverable(pl, r) for r in range(3)]
+    assert sum(counts) == 100
+    assert counts == [sum(1 for p in range(pl.psi_pad)
+                          if P.locate(pl, p)[1] == r and not P.is_padding(pl, p))
+                      for r in range(3)]
+    assert P.lost_rank_unrecoverable(P.make_plan(100, 3, 0, 10), 1) == 0
+
+
+def test_reshard_keeps_every_real_element():
+    rng = np.random.default_rng(30)
+    units = [37, 63, 5]
+    a = P.make_plan(105, 3, 3, 10, align=4, unit_elems=units)
+    b = P.make_plan(105, 8, 1, 7, align=1, unit_elems=units)
+    x = rng.standard_normal(a.nd * a.S).astype(np.float32)
+    pad_a = np.array([P.is_padding(a, p) for p in range(a.psi_pad)])
+    x[ST.logical_to_storage(a, pad_a.astype(np.float32)) > 0] = 0
+    y = ST.reshard(a, x, b)
+    for p in range(b.psi_pad):
+        u, o, off, j = P.locate(b, p)
+        if j < units[u]:
+            pa = a.unit_base[u] + j          # same unit, same index under plan a
+            _, oa, offa, _ = P.locate(a, pa)
+            assert y[o * b.S + off] == x[oa * a.S + offa]
+        else:
+            assert y[o * b.S + off] == 0
+    assert np.array_equal(ST.reshard(b, y, a), x)

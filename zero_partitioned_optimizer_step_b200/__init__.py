@@ -27,7 +27,8 @@ ZERO_OK, ZERO_EINVAL, ZERO_ENOMEM, ZERO_ECUDA, ZERO_ESTATE, ZERO_ETIMEOUT = rang
  ZERO_Q_BUCKET_END, ZERO_Q_OWNER, ZERO_Q_OWNER_OFFSET, ZERO_Q_MEM_BYTES_PER_RANK,
  ZERO_Q_WORKSPACE_BYTES, ZERO_Q_LIVE_UNITS, ZERO_Q_PEAK_LIVE_UNITS,
  ZERO_Q_PEAK_LIVE_BYTES, ZERO_Q_IS_LIVE, ZERO_Q_MAX_LIVE, ZERO_Q_ALIGN,
- ZERO_Q_BUCKET_ELEMS) = range(26)
+ ZERO_Q_BUCKET_ELEMS, ZERO_Q_STATE_REPLICAS, ZERO_Q_GRAD_REPLICAS, ZERO_Q_PARAM_REPLICAS,
+ ZERO_Q_LOST_RANK_UNRECOVERABLE) = range(30)
 
 # accounting kinds (zero_bytes_kind_t) and flags
 (ZERO_BYTES_COMM_ELEMS_PER_RANK, ZERO_BYTES_COMM_PER_RANK, ZERO_BYTES_HBM_STEP,
@@ -109,6 +110,8 @@ def lib():
         L.zero_bytes_moved.argtypes = [vp, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(u64)]
         L.zero_step_kernel.restype = st
         L.zero_step_kernel.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)]
+        L.zero_reshard.restype = st
+        L.zero_reshard.argtypes = [vp, vp, vp, vp, ctypes.c_uint32, vp]
         L.zero_stream_status.restype = st
         L.zero_stream_status.argtypes = [vp]
         L.zero_status_str.restype = ctypes.c_char_p
@@ -352,6 +355,16 @@ def zero_stream_status(stream=None):
     """Synchronise the stream; raise ZeroError(ZERO_ETIMEOUT) if a bounded
     wait in the bulk-copy kernel gave up since the last check."""
     _check(lib().zero_stream_status(_stream(stream)))
+
+
+def zero_reshard(from_plan, src, to_plan, dst, stream=None):
+    """Copy one owner-storage state array (fp32 or bf16 tensor) from
+    `from_plan`'s layout to `to_plan`'s (same units, other Nd or padding)."""
+    import torch
+    if src.dtype != dst.dtype or src.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("src and dst must both be float32 or both bfloat16")
+    _check(lib().zero_reshard(from_plan.handle, _ptr(src, None, "src"), to_plan.handle,
+                              _ptr(dst, None, "dst"), src.element_size(), _stream(stream)))
 
 
 def workspace_for(plan, device="cuda"):

@@ -157,6 +157,21 @@ ZERO_API zero_status_t zero_plan_query(const zero_plan_t *p, zero_query_t what,
         case ZERO_Q_MAX_LIVE: *out = p->max_live; return ZERO_OK;
         case ZERO_Q_ALIGN: *out = p->align; return ZERO_OK;
         case ZERO_Q_BUCKET_ELEMS: *out = p->bucket_elems; return ZERO_OK;
+        case ZERO_Q_STATE_REPLICAS: *out = p->stage == 0 ? p->nd : 1; return ZERO_OK;
+        case ZERO_Q_GRAD_REPLICAS: *out = p->stage <= 1 ? p->nd : 1; return ZERO_OK;
+        case ZERO_Q_PARAM_REPLICAS: *out = p->stage <= 2 ? p->nd : 1; return ZERO_OK;
+        case ZERO_Q_LOST_RANK_UNRECOVERABLE: {
+            if (idx >= p->nd) return set_error(ZERO_EINVAL, "zero_plan_query: rank out of range");
+            uint64_t lost = 0;
+            if (p->stage != 0 || p->nd == 1) {
+                for (size_t u = 0; u < nu; ++u) {
+                    const uint64_t lo = idx * p->unit_shard[u];
+                    if (p->unit_len[u] > lo) lost += std::min(p->unit_shard[u], p->unit_len[u] - lo);
+                }
+            }
+            *out = lost;
+            return ZERO_OK;
+        }
         case ZERO_Q_UNIT_LEN:
         case ZERO_Q_UNIT_PAD:
         case ZERO_Q_UNIT_SHARD:

@@ -770,3 +770,65 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     }
     return ZERO_OK;
 }
+
+// ------------------------------------------------------------- resharding
+namespace {
+
+// K4: one unit's elements from owner storage under plan A to owner storage
+// under plan B (same unit lengths, other Nd or padding).  Thread per
+// destination element q of the unit's slices: owner o' = q / s'_u,
+// logical j = o' * s'_u + (q mod s'_u); j >= len_u is padding (zero).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) k_reshard(const T *src, uint64_t S_a, uint64_t off_a, uint64_t s_a,
+                                                     T *dst, uint64_t S_b, uint64_t off_b, uint64_t s_b,
+                                                     uint32_t nd_b, uint64_t len) {
+    const uint64_t n = uint64_t(nd_b) * s_b;
+    const uint64_t stride = uint64_t(gridDim.x) * kThreads;
+    for (uint64_t q = uint64_t(blockIdx.x) * kThreads + threadIdx.x; q < n; q += stride) {
+        const uint64_t ob = q / s_b, i = q - ob * s_b;
+        const uint64_t j = q;  // logical index inside the unit (ob * s_b + i)
+        T val = T(0);
+        if (j < len) {
+            const uint64_t oa = j / s_a;
+            val = src[oa * S_a + off_a + (j - oa * s_a)];
+        }
+        dst[ob * S_b + off_b + i] = val;
+    }
+}
+
+}  // namespace
+
+ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, const zero_plan_t *to, void *dst,
+                                    uint32_t elem_bytes, void *stream_) {
+    zero_detail::clear_error();
+    if (!from || !to || !src || !dst) return set_error(ZERO_EINVAL, "zero_reshard: NULL argument");
+    if (elem_bytes != 2 && elem_bytes != 4)
+        return set_error(ZERO_EINVAL, "zero_reshard: elem_bytes must be 2 (bf16) or 4 (fp32)");
+    if (from->unit_len != to->unit_len)
+        return set_error(ZERO_EINVAL, "zero_reshard: the two plans must have the same unit lengths");
+    if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % elem_bytes)
+        return set_error(ZERO_EINVAL, "zero_reshard: buffers must be aligned to the element size");
+    cudaError_t pre = cudaPeekAtLastError();
+    if (pre != cudaSuccess)
+        return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_reshard: ") +
+                                         cudaGetErrorString(pre));
+    DeviceShapes shapes;
+    zero_status_t st = device_shapes(&shapes);
+    if (st != ZERO_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    for (size_t u = 0; u < to->unit_len.size(); ++u) {
+        const uint64_t n = uint64_t(to->nd) * to->unit_shard[u];
+        const uint32_t grid = uint32_t(std::min<uint64_t>((n + kThreads - 1) / kThreads, uint64_t(shapes.sms) * 8));
+        if (elem_bytes == 4)
+            k_reshard<uint32_t><<<grid, kThreads, 0, stream>>>(
+                static_cast<const uint32_t *>(src), from->S, from->unit_offset[u], from->unit_shard[u],
+                static_cast<uint32_t *>(dst), to->S, to->unit_offset[u], to->unit_shard[u], to->nd, to->unit_len[u]);
+        else
+            k_reshard<uint16_t><<<grid, kThreads, 0, stream>>>(
+                static_cast<const uint16_t *>(src), from->S, from->unit_offset[u], from->unit_shard[u],
+                static_cast<uint16_t *>(dst), to->S, to->unit_offset[u], to->unit_shard[u], to->nd, to->unit_len[u]);
+        st = check_launch("zero_reshard launch");
+        if (st != ZERO_OK) return st;
+    }
+    return ZERO_OK;
+}
