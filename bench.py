@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step replayed as a CUDA graph (workloads without layer gathers)")
     ap.add_argument("--psi", type=int, default=None,
                     help="override the parameter count (flat single-unit workloads only)")
     ap.add_argument("--shard", type=int, default=None,
@@ -263,6 +265,15 @@ class Workload:
                                 if owner >= 0 else cfg["psi"])
         self.nb = self.lp.n_buckets
 
+    def make_graph(self):
+        """The step captured as CUDA graphs (zero_partitioned_optimizer_step_b200.graph)."""
+        from zero_partitioned_optimizer_step_b200.graph import StepGraph
+        if self.layer is not None:
+            raise SystemExit("--graph: the stage-3 layer gathers are not captured")
+        return StepGraph(self.lp, self.G, self.w, self.m, self.v, self.params, self.adam,
+                         grad_norm_sq=self.norm, overflow=self.ovf, workspace=self.ws,
+                         owner_view=self.owner)
+
     def rebucket(self, bucket_elems):
         """Same buffers, a new plan with another bucket size."""
         cfg = self.cfg
@@ -382,12 +393,21 @@ def run_ours(args, cfg, rank, world, dist):
     wl = Workload(cfg, dev)
     stream = torch.cuda.current_stream(dev)
     # warm-up (also builds the per-device launch grid)
-    for t in range(1, args.warmup + 1):
+    t = 1
+    for _ in range(args.warmup):
         wl.step(t, stream)
+        t += 1
+    sg = None
+    if args.graph:
+        sg = wl.make_graph()
+        for _ in range(args.warmup):
+            sg.replay(t)
+            t += 1
     torch.cuda.synchronize()
 
+    n_ev = args.steps if sg is None else min(args.steps, 50)
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(wl.nb + 1)]
-              for _ in range(args.steps)]
+              for _ in range(n_ev)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index).start()
@@ -396,19 +416,27 @@ def run_ours(args, cfg, rank, world, dist):
         dist.barrier()
     torch.cuda.synchronize()
     start.record(stream)
-    t0 = args.warmup + 1
+    t0 = t
     for k in range(args.steps):
-        wl.step(t0 + k, stream, events[k])
+        if sg is not None:
+            sg.replay(t0 + k)
+        else:
+            wl.step(t0 + k, stream, events[k])
     end.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
     elapsed = start.elapsed_time(end) / 1e3
+    if sg is not None:
+        # the kernel's own rate, from eager steps with an event per bucket
+        for k in range(n_ev):
+            wl.step(t0 + args.steps + k, stream, events[k])
+        torch.cuda.synchronize()
     # dominant kernel: the fused bucket kernel, timed per launch
     k1_time = 0.0
     k1_elems = 0
-    for k in range(args.steps):
+    for k in range(n_ev):
         for b in range(wl.nb):
             if wl.bucket_elems(b) == 0:
                 continue
@@ -420,10 +448,12 @@ def run_ours(args, cfg, rank, world, dist):
     # every step, the step, the norm and overflow flag read back every step
     e2e = None
     if not args.no_e2e:
-        e2e = _e2e(args, wl, stream, dev, world, dist, t0 + args.steps)
+        e2e = _e2e(args, wl, stream, dev, world, dist, t0 + args.steps + n_ev)
     if rank != 0:
         return None
-    return _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e)
+    res = _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=n_ev)
+    res["config"]["graph"] = sg is not None
+    return res
 
 
 def _e2e(args, wl, stream, dev, world, dist, t_first):
@@ -452,12 +482,12 @@ def _e2e(args, wl, stream, dev, world, dist, t_first):
             "d2h_bytes_per_step": 8 + 4, "steps": e2e_steps}
 
 
-def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e):
+def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=None):
     peak, peak_kind = measured_peak()
     per_elem = wl.step_bytes / wl.elems
     k1_bytes = per_elem * k1_elems
     achieved = k1_bytes / k1_time / 1e9
-    n_launch = args.steps * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
+    n_launch = (n_ev or args.steps) * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
     tr = (k1_traffic_per_elem() if (args.config == "c2" and args.psi is None
                                     and wl.Z.zero_step_kernel(wl.lp, wl.owner) == "k_step_tma") else None)
     kname = wl.Z.zero_step_kernel(wl.lp, wl.owner)
@@ -530,11 +560,30 @@ def run_sweep(args, rank, world, dist):
                 a.no_cpu_baseline = True
                 res = _report(a, cfg, wl, world, elapsed, k1_time, k1_elems, None, None)
                 res["config"]["bucket_mb"] = mb
+                if args.graph:
+                    sg = wl.make_graph()
+                    tg = 10 ** 6
+                    for _ in range(2):
+                        sg.replay(tg)
+                        tg += 1
+                    torch.cuda.synchronize()
+                    s0.record(stream)
+                    for _ in range(args.steps):
+                        sg.replay(tg)
+                        tg += 1
+                    s1.record(stream)
+                    torch.cuda.synchronize()
+                    eg = s0.elapsed_time(s1) / 1e3
+                    res["graph"] = {"value": job_value(world, wl.params_per_step, args.steps, eg),
+                                    "ms_per_step": eg / args.steps * 1e3,
+                                    "hbm_gbs": wl.step_bytes / (eg / args.steps) / 1e9}
+                    del sg
                 f.write(json.dumps(res) + "\n")
                 f.flush()
                 print(json.dumps({"nd": nd, "mb": mb, "value": res["value"],
                                   "step_gbs": res["hbm_gbs"], "k1_gbs": res["roofline"]["achieved"],
-                                  "k1_frac": res["roofline"]["frac"]}), flush=True)
+                                  "k1_frac": res["roofline"]["frac"],
+                                  "graph_value": (res.get("graph") or {}).get("value")}), flush=True)
             del wl
             torch.cuda.empty_cache()
 

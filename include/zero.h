@@ -58,6 +58,9 @@
  * shared-memory ring fits Nd rows, else in the 16-byte-vector load kernel;
  * unaligned heads and tails in a scalar kernel.  All give identical results.
  * The environment variable ZERO_STEP_KERNEL=ldg|tma overrides the choice.
+ * ZERO_TEST_STALL_PRODUCER=<cta> exists only to test failure detection: that
+ * CTA of the bulk-copy kernel loads nothing, its waits run out after 2 s, and
+ * zero_stream_status() reports ZERO_ETIMEOUT (outputs of that step invalid).
  * Threads.  A plan may be shared by threads for zero_step*() and queries;
  * zero_gather_layer()/zero_release_layer() serialise on the plan internally.
  */
@@ -203,7 +206,20 @@ typedef struct zero_bufs {
                               overflow is set; caller-owned */
     uint64_t workspace_bytes;
     int32_t owner_view;    /* -1: all Nd ranks; o in [0,Nd): rank o only */
+    const void *adam_consts; /* optional device pointer to the 9 fp32 step
+                              constants of zero_adam_consts(); when set the
+                              kernels read them from there instead of from
+                              adam and t, so a step captured in a CUDA graph
+                              can be replayed for a new t by refreshing this
+                              buffer (e.g. by a captured copy from pinned
+                              host memory).  16-byte aligned. */
 } zero_bufs_t;
+
+/* The nine fp32 constants one step uses, in this order: grad_scale, beta1,
+ * beta2, eps, 1-beta1, 1-beta2, lr/(1-beta1^t), 1/sqrt(1-beta2^t),
+ * 1-lr*weight_decay (each computed in double and rounded once).  Host only.
+ * ZERO_EINVAL: NULL argument or t = 0. */
+zero_status_t zero_adam_consts(const zero_adam_t *adam, uint64_t t, float out[9]);
 
 /* One full step: every bucket in order, then (if asked) the norm/overflow.
  * Source: [MM] section "但 GPU 只存四分之一…" (gradients are split back to

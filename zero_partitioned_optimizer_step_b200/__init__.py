@@ -68,7 +68,7 @@ class _Bufs(ctypes.Structure):
                 ("param_stride", ctypes.c_uint64), ("reduced_grad", ctypes.c_void_p),
                 ("grad_norm_sq", ctypes.c_void_p), ("overflow", ctypes.c_void_p),
                 ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
-                ("owner_view", ctypes.c_int32)]
+                ("owner_view", ctypes.c_int32), ("adam_consts", ctypes.c_void_p)]
 
 
 _LIB = None
@@ -112,6 +112,8 @@ def lib():
         L.zero_step_kernel.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)]
         L.zero_reshard.restype = st
         L.zero_reshard.argtypes = [vp, vp, vp, vp, ctypes.c_uint32, vp]
+        L.zero_adam_consts.restype = st
+        L.zero_adam_consts.argtypes = [ctypes.POINTER(_Adam), u64, vp]
         L.zero_stream_status.restype = st
         L.zero_stream_status.argtypes = [vp]
         L.zero_status_str.restype = ctypes.c_char_p
@@ -260,7 +262,7 @@ def _row_stride(t, default):
 
 def make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, reduced_grad=None,
               grad_norm_sq=None, overflow=None, workspace=None, owner_view=-1,
-              grad_stride=None, param_stride=None):
+              grad_stride=None, param_stride=None, adam_consts=None):
     import torch
     b = _Bufs()
     b.grads = _ptr(grads, torch.bfloat16, "grads")
@@ -278,6 +280,7 @@ def make_bufs(plan, grads, master, exp_avg, exp_avg_sq, params, reduced_grad=Non
     b.workspace = _ptr(workspace, None, "workspace")
     b.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     b.owner_view = int(owner_view)
+    b.adam_consts = _ptr(adam_consts, torch.float32, "adam_consts")
     return b
 
 
@@ -349,6 +352,16 @@ def zero_step_kernel(plan, owner_view=-1):
     out = ctypes.c_uint32()
     _check(lib().zero_step_kernel(plan.handle, int(owner_view), ctypes.byref(out)))
     return "k_step_tma" if out.value == ZERO_KERNEL_BULK_COPY else "k_step_vec8"
+
+
+def zero_adam_consts(adam, t, out):
+    """Fill `out` (a float32 tensor of >= 9 elements on the host) with step t's
+    nine fp32 constants."""
+    import torch
+    if out.dtype != torch.float32 or out.numel() < 9 or out.is_cuda or not out.is_contiguous():
+        raise ValueError("out must be a contiguous host float32 tensor of >= 9 elements")
+    _check(lib().zero_adam_consts(ctypes.byref(make_adam(adam)), int(t),
+                                  ctypes.c_void_p(out.data_ptr())))
 
 
 def zero_stream_status(stream=None):

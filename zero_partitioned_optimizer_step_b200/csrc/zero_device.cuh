@@ -34,6 +34,7 @@ struct StepArgs {
     uint64_t shard, jump, p_jump;
     uint64_t j0, j1;
     AdamConsts c;
+    const AdamConsts *cdev;  // if set, the constants are read from device memory
     double *ws_norm;
     uint32_t *ws_bad;
     int ws_mode;  // 0: no norm; 1: add this launch's per-CTA partials to the slots
@@ -63,6 +64,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ bool not_finite(float x) {
     return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
+}
+
+// The Adam constants of a launch: from device memory when the caller
+// supplied them there (so that a captured graph can be replayed for a new t),
+// else the launch arguments.
+__device__ __forceinline__ AdamConsts consts_of(const StepArgs &a) {
+    return a.cdev ? *a.cdev : a.c;
 }
 
 // Textbook Adam on one element with decoupled weight decay, every operation

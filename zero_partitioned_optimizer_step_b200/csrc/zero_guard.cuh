@@ -117,6 +117,7 @@ template <int VEC, bool OWNER_MAP>
 __global__ void __launch_bounds__(kThreads) k_apply(const StepArgs a, const GuardWord *gw) {
     const GuardWord g = *gw;
     if (g.skip) return;
+    const AdamConsts C = zero_dev::consts_of(a);
     const uint64_t n = (a.j1 - a.j0) / VEC;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
     for (uint64_t vi = uint64_t(blockIdx.x) * kThreads + threadIdx.x; vi < n; vi += stride) {
@@ -139,7 +140,7 @@ __global__ void __launch_bounds__(kThreads) k_apply(const StepArgs a, const Guar
                 v[4 * h] = v4.x; v[4 * h + 1] = v4.y; v[4 * h + 2] = v4.z; v[4 * h + 3] = v4.w;
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) zero_dev::adam1c(s[e], g.coef, a.c, w[e], m[e], v[e]);
+            for (int e = 0; e < 8; ++e) zero_dev::adam1c(s[e], g.coef, C, w[e], m[e], v[e]);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 __stcs(reinterpret_cast<float4 *>(a.w + si) + h,
@@ -158,7 +159,7 @@ __global__ void __launch_bounds__(kThreads) k_apply(const StepArgs a, const Guar
                 __stcs(reinterpret_cast<uint4 *>(a.params + pi + uint64_t(r) * a.param_stride), pk);
         } else {
             float w = a.w[si], m = a.m[si], v = a.v[si];
-            zero_dev::adam1c(a.red[si], g.coef, a.c, w, m, v);
+            zero_dev::adam1c(a.red[si], g.coef, C, w, m, v);
             a.w[si] = w;
             a.m[si] = m;
             a.v[si] = v;

@@ -60,6 +60,7 @@ using namespace zero_dev;
 // per SM the register budget is sized for.
 template <bool OWNER_MAP, int RB, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB) k_step_vec8(const StepArgs a) {
+    const AdamConsts C = consts_of(a);
     const uint64_t nvec = (a.j1 - a.j0) >> 3;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
     uint64_t vi = uint64_t(blockIdx.x) * kThreads + threadIdx.x;
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, MINB) k_step_vec8(const StepArgs a) 
         float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
         float vv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) adam1(s[e], a.c, wv[e], mv[e], vv[e]);
+        for (int e = 0; e < 8; ++e) adam1(s[e], C, wv[e], mv[e], vv[e]);
 
         __stcs(reinterpret_cast<float4 *>(a.w + si), make_float4(wv[0], wv[1], wv[2], wv[3]));
         __stcs(reinterpret_cast<float4 *>(a.w + si + 4), make_float4(wv[4], wv[5], wv[6], wv[7]));
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, MINB) k_step_vec8(const StepArgs a) 
 // K1, scalar path: any alignment (A not a multiple of 8, odd strides, bucket
 // heads and tails).  Same arithmetic, one element per thread and iteration.
 __global__ void __launch_bounds__(kThreads) k_step_scalar(const StepArgs a) {
+    const AdamConsts C = consts_of(a);
     const uint64_t n = a.j1 - a.j0;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
     double acc = 0.0;
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kThreads) k_step_scalar(const StepArgs a) {
         }
         if (a.red) a.red[si] = s;
         float w = a.w[si], m = a.m[si], v = a.v[si];
-        adam1(s, a.c, w, m, v);
+        adam1(s, C, w, m, v);
         a.w[si] = w;
         a.m[si] = m;
         a.v[si] = v;
@@ -374,6 +376,14 @@ bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, zero_tma::Ring *
     if (force_v == 2 || force_v == 4 || force_v == 8) vw = uint32_t(force_v);
     zero_tma::Ring q = ring_for(nd, tile, 0, groups);
     q.vw = vw;
+    // ZERO_TEST_STALL_PRODUCER=<cta>: that CTA's producer issues nothing, so
+    // its consumers' bounded waits run out (tests the ZERO_ETIMEOUT path)
+    q.stall_cta = 0xffffffffu;
+    if (const char *e = std::getenv("ZERO_TEST_STALL_PRODUCER")) {
+        char *end = nullptr;
+        const unsigned long v = std::strtoul(e, &end, 10);
+        if (end != e && v < 0xffffffffu) q.stall_cta = uint32_t(v);
+    }
     uint64_t ns = std::min<uint64_t>(budget / q.stage_bytes, stages);
     ns -= ns % groups;  // every stage belongs to one group
     if (ns < 2) return false;
@@ -477,7 +487,7 @@ zero_status_t validate_step(const zero_plan_t *p, const zero_bufs_t *b, const ze
         if (!q) return set_error(ZERO_EINVAL, "zero_step: grads, master, exp_avg, exp_avg_sq and params are required");
         if (!aligned16(q)) return set_error(ZERO_EINVAL, "zero_step: device pointers must be 16-byte aligned");
     }
-    const void *opt[] = {b->reduced_grad, b->grad_norm_sq, b->overflow, b->workspace};
+    const void *opt[] = {b->reduced_grad, b->grad_norm_sq, b->overflow, b->workspace, b->adam_consts};
     for (const void *q : opt)
         if (q && !aligned16(q)) return set_error(ZERO_EINVAL, "zero_step: device pointers must be 16-byte aligned");
     const bool owner = b->owner_view >= 0;
@@ -506,6 +516,7 @@ StepArgs base_args(const zero_plan_t *p, const zero_bufs_t *b, const zero_adam_t
     a.n_prow = replicas ? p->nd : 1;
     a.nd = p->nd;
     a.c = make_consts(*adam, t);
+    a.cdev = static_cast<const AdamConsts *>(b->adam_consts);
     auto *ws = static_cast<unsigned char *>(b->workspace);
     a.ws_norm = reinterpret_cast<double *>(ws);
     a.ws_bad = reinterpret_cast<uint32_t *>(ws + 8ull * zero_detail::kMaxSlots);
@@ -830,5 +841,15 @@ ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, co
         st = check_launch("zero_reshard launch");
         if (st != ZERO_OK) return st;
     }
+    return ZERO_OK;
+}
+
+ZERO_API zero_status_t zero_adam_consts(const zero_adam_t *adam, uint64_t t, float out[9]) {
+    zero_detail::clear_error();
+    if (!adam || !out) return set_error(ZERO_EINVAL, "zero_adam_consts: NULL argument");
+    if (t == 0) return set_error(ZERO_EINVAL, "zero_adam_consts: t must be >= 1");
+    static_assert(sizeof(AdamConsts) == 9 * sizeof(float), "nine packed fp32 constants");
+    const AdamConsts c = make_consts(*adam, t);
+    std::memcpy(out, &c, sizeof c);
     return ZERO_OK;
 }

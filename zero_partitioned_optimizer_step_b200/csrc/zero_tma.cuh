@@ -49,6 +49,8 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 // `tile` bf16 at offset 0, then w, m, v (fp32).  `vw` is the per-thread
 // vector width the kernel was instantiated with.
 struct Ring {
+    uint32_t stall_cta;  // test of the bounded waits: this CTA's producer issues
+                         // nothing (0xffffffff: none)
     uint32_t vw;
     uint32_t tile;
     uint32_t stages;  // a multiple of groups
@@ -256,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
+        if (blockIdx.x == ring.stall_cta) return;  // consumers' waits run out
         uint32_t k = 0;
         for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
             const uint32_t s = k % NS;
@@ -300,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
     }
 
     // ---------------------------------------------------------- consumers
+    const AdamConsts C = zero_dev::consts_of(a);
     // Group g takes the CTA's tiles k = g, g + GROUPS, ..., so one group's
     // per-tile latency overlaps the other's.
     const int ct = threadIdx.x - 32;
@@ -349,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
                 const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
                 if (a.red) stg_f32<VW>(a.red + si, sum);
 #pragma unroll
-                for (int e = 0; e < VW; ++e) zero_dev::adam1(sum[e], a.c, wv[e], mv[e], vq[e]);
+                for (int e = 0; e < VW; ++e) zero_dev::adam1(sum[e], C, wv[e], mv[e], vq[e]);
                 stg_f32<VW>(a.w + si, wv);
                 stg_f32<VW>(a.m + si, mv);
                 stg_f32<VW>(a.v + si, vq);
