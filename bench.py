@@ -1,8 +1,10 @@
 """Benchmark of the ZeRO partitioned optimizer step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config c2] [--nd ND --bucket-mb MB]   # c5 points
-                    [--sweep OUT.jsonl]                      # whole c5 grid
+                    [--config gpt2_small|toy|stage3_1p3b|owner_7p5b|sweep]
+                    [--nd ND --bucket-mb MB]                 # one bucket-sweep point
+                    [--sweep OUT.jsonl]                      # the whole bucket sweep
+                    [--graph]                                # replay the step as a CUDA graph
 
 One step = the whole hot path over one batch of gradients: for every bucket,
 the fused reduce-scatter + owner Adam + all-gather kernel, then the
@@ -58,12 +60,13 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5"])
+    ap.add_argument("--config", default="gpt2_small",
+                    choices=["toy", "gpt2_small", "stage3_1p3b", "owner_7p5b", "sweep"])
     ap.add_argument("--nd", type=int, default=None,
                     help="logical ranks (bucket sweep point: default 64; other workloads: "
                          "override their Nd)")
     ap.add_argument("--bucket-mb", type=int, default=64)
-    ap.add_argument("--sweep", default=None, help="write the c5 grid as JSON lines here")
+    ap.add_argument("--sweep", default=None, help="write the bucket sweep grid as JSON lines here")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -79,9 +82,9 @@ def parse_args():
 
 
 def get_cfg(args):
-    from zero_partitioned_optimizer_step_b200.configs import CONFIGS, c5_config
-    if args.config == "c5":
-        cfg = c5_config(args.nd or 64, args.bucket_mb)
+    from zero_partitioned_optimizer_step_b200.configs import CONFIGS, sweep_config
+    if args.config == "sweep":
+        cfg = sweep_config(args.nd or 64, args.bucket_mb)
     else:
         cfg = dict(CONFIGS[args.config])
         if args.nd is not None:
@@ -230,13 +233,13 @@ class Workload:
         if owner >= 0:
             n = self.S
             real = min(max(cfg["psi"] - owner * n, 0), n)
-            self.G = inputs.grads(nd, [real], [n], cfg["sigma"], cfg["id"], 1, device)
-            self.w = inputs.master_logical([real], [n], cfg["id"], device)
+            self.G = inputs.grads(nd, [real], [n], cfg["sigma"], cfg["seed_id"], 1, device)
+            self.w = inputs.master_logical([real], [n], cfg["seed_id"], device)
         else:
             n = nd * self.S
-            self.G = inputs.grads(nd, unit_len, unit_pad, cfg["sigma"], cfg["id"], 1, device,
+            self.G = inputs.grads(nd, unit_len, unit_pad, cfg["sigma"], cfg["seed_id"], 1, device,
                                   outlier_frac=cfg["outlier_frac"])
-            w_log = inputs.master_logical(unit_len, unit_pad, cfg["id"], device)
+            w_log = inputs.master_logical(unit_len, unit_pad, cfg["seed_id"], device)
             self.w = torch.empty(n, dtype=torch.float32, device=device)
             for o in range(nd):
                 for (ln, P, s, U, O) in self.units:
@@ -359,10 +362,10 @@ def run_reference(args, cfg):
     from zero_partitioned_optimizer_step_b200 import inputs
     nd = cfg["nd"]
     n = 1 << 22
-    G = inputs.grads(nd, [n], [n], cfg["sigma"], cfg["id"], 1, "cpu",
+    G = inputs.grads(nd, [n], [n], cfg["sigma"], cfg["seed_id"], 1, "cpu",
                      outlier_frac=cfg["outlier_frac"])
     G = G.view(torch.int16).numpy().view(np.uint16)
-    w = inputs.master_logical([n], [n], cfg["id"], "cpu").numpy()
+    w = inputs.master_logical([n], [n], cfg["seed_id"], "cpu").numpy()
     m = np.zeros(n, np.float32)
     v = np.zeros(n, np.float32)
     adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
@@ -488,7 +491,7 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=Non
     k1_bytes = per_elem * k1_elems
     achieved = k1_bytes / k1_time / 1e9
     n_launch = (n_ev or args.steps) * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
-    tr = (k1_traffic_per_elem() if (args.config == "c2" and args.psi is None
+    tr = (k1_traffic_per_elem() if (args.config == "gpt2_small" and args.psi is None
                                     and wl.Z.zero_step_kernel(wl.lp, wl.owner) == "k_step_tma") else None)
     kname = wl.Z.zero_step_kernel(wl.lp, wl.owner)
     roof = {"kernel": kname + " (fused reduce-scatter + Adam + all-gather, one bucket)",
@@ -525,12 +528,12 @@ def run_sweep(args, rank, world, dist):
     """The bucket-size sweep (5e8 params): for each Nd one set of buffers, then
     every bucket size from 1 MB to 512 MB of one rank's bf16 gradient."""
     import torch
-    from zero_partitioned_optimizer_step_b200.configs import c5_config
+    from zero_partitioned_optimizer_step_b200.configs import sweep_config
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     with open(args.sweep, "w") as f:
         for nd in (2, 4, 8, 16, 64):
-            wl = Workload(c5_config(nd, 1), dev)
+            wl = Workload(sweep_config(nd, 1), dev)
             for mb in (1, 2, 4, 8, 16, 32, 64, 128, 256, 512):
                 wl.rebucket(mb << 19)
                 cfg = dict(wl.cfg, workload="bucket sweep psi=5e8, Nd=%d, %d MB buckets" % (nd, mb))
@@ -556,7 +559,7 @@ def run_sweep(args, rank, world, dist):
                               for k in range(args.steps) for b in range(wl.nb))
                 k1_elems = args.steps * sum(wl.bucket_elems(b) for b in range(wl.nb))
                 a = argparse.Namespace(**vars(args))
-                a.config = "c5"
+                a.config = "sweep"
                 a.no_cpu_baseline = True
                 res = _report(a, cfg, wl, world, elapsed, k1_time, k1_elems, None, None)
                 res["config"]["bucket_mb"] = mb

@@ -95,16 +95,16 @@ def test_plan_bit_exact_to_oracle_bruteforce():
     assert n == 64 * 7 * 3
 
 
-@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4", "c5"])
+@pytest.mark.parametrize("name", ["toy", "gpt2_small", "stage3_1p3b", "owner_7p5b", "sweep"])
 def test_plan_bit_exact_to_oracle_configs(name):
-    if name == "c1":
+    if name == "toy":
         check_against_oracle(65536, 4, 2, 4096, 64, None)
-    elif name == "c2":
+    elif name == "gpt2_small":
         check_against_oracle(124_439_808, 8, 2, 25_000_000, 64, None, every_index=False)
-    elif name == "c3":
+    elif name == "stage3_1p3b":
         units = [107_120_640] + [50_358_272] * 24 + [4096]
         check_against_oracle(sum(units), 16, 3, 1 << 27, 64, units, every_index=False)
-    elif name == "c4":
+    elif name == "owner_7p5b":
         check_against_oracle(7_500_000_000, 64, 2, 25_000_000, 64, None, every_index=False)
     else:
         for nd in (2, 4, 8, 16, 64):

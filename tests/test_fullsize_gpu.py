@@ -10,7 +10,7 @@ import torch
 
 import zero_partitioned_optimizer_step_b200 as Z
 from zero_partitioned_optimizer_step_b200 import inputs
-from zero_partitioned_optimizer_step_b200.configs import ADAM, CONFIGS, c5_config
+from zero_partitioned_optimizer_step_b200.configs import ADAM, CONFIGS, sweep_config
 from oracle import core
 from oracle import plan as OP
 from zero_cases import RTOL_NORM, RTOL_STATE, BF16_ULP, bf16_ulp_check, f32_rel_check, u16
@@ -59,7 +59,7 @@ class WindowRun:
             self.sidx = self.cols
             real = min(max(cfg["psi"] - lo, 0), n)   # single unit: padding at the end
             self.g_units = ([real], [n]) if real < n else ([n], [n])
-            self.w = inputs.master_logical([n], [n], cfg["id"], dev)
+            self.w = inputs.master_logical([n], [n], cfg["seed_id"], dev)
             if real < n:
                 self.w[real:].zero_()
         else:
@@ -74,7 +74,7 @@ class WindowRun:
                 ranges += [(x, x + WIN) for x in rnd.integers(0, op.psi_pad - WIN, 4)]
             self.cols = _ranges_to_cols(ranges, op.psi_pad)
             self.sidx = OP.storage_index(op, self.cols)
-            w_log = inputs.master_logical(op.unit_len, op.unit_pad, cfg["id"], dev)
+            w_log = inputs.master_logical(op.unit_len, op.unit_pad, cfg["seed_id"], dev)
             self.w = torch.empty(op.nd * op.S, dtype=torch.float32, device=dev)
             for o in range(op.nd):
                 for u in range(len(op.unit_pad)):
@@ -106,11 +106,11 @@ class WindowRun:
             real, n = self.g_units[0][0], self.g_units[1][0]
             if self.G is None:
                 self.G = torch.empty((cfg["nd"], n), dtype=torch.bfloat16, device="cuda")
-            return inputs.grads(cfg["nd"], [real], [n], cfg["sigma"], cfg["id"], t, "cuda",
+            return inputs.grads(cfg["nd"], [real], [n], cfg["sigma"], cfg["seed_id"], t, "cuda",
                                 cfg["outlier_frac"], out=self.G)
         if self.G is None:
             self.G = torch.empty((cfg["nd"], self.op.psi_pad), dtype=torch.bfloat16, device="cuda")
-        return inputs.grads(cfg["nd"], self.op.unit_len, self.op.unit_pad, cfg["sigma"], cfg["id"],
+        return inputs.grads(cfg["nd"], self.op.unit_len, self.op.unit_pad, cfg["sigma"], cfg["seed_id"],
                             t, "cuda", cfg["outlier_frac"], out=self.G)
 
     def step(self, t, full_norm=False):
@@ -160,13 +160,13 @@ class WindowRun:
 
 
 def test_c2_gpt2_small_stage2_ten_steps():
-    r = WindowRun(CONFIGS["c2"])
-    for t in range(1, CONFIGS["c2"]["steps"] + 1):
+    r = WindowRun(CONFIGS["gpt2_small"])
+    for t in range(1, CONFIGS["gpt2_small"]["steps"] + 1):
         r.step(t, full_norm=(t == 1))
 
 
 def test_c3_stage3_layerwise_five_steps():
-    cfg = CONFIGS["c3"]
+    cfg = CONFIGS["stage3_1p3b"]
     r = WindowRun(cfg)
     n_units = len(cfg["units"])
     for t in range(1, cfg["steps"] + 1):
@@ -176,7 +176,7 @@ def test_c3_stage3_layerwise_five_steps():
 
 
 def test_c4_single_owner_of_7p5b():
-    cfg = CONFIGS["c4"]
+    cfg = CONFIGS["owner_7p5b"]
     r = WindowRun(cfg)
     for t in range(1, cfg["steps"] + 1):
         r.step(t)
@@ -192,7 +192,7 @@ def test_c4_single_owner_of_7p5b():
 
 @pytest.mark.parametrize("nd,mb", [(2, 1), (2, 512), (16, 64), (64, 1), (64, 512)])
 def test_c5_bucket_sweep_points(nd, mb):
-    cfg = c5_config(nd, mb)
+    cfg = sweep_config(nd, mb)
     r = WindowRun(cfg, seed=nd * 1000 + mb)
     r.step(1)
     r.step(2)

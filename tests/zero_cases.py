@@ -12,7 +12,7 @@ from oracle import step as ST
 
 FLT_MIN = np.float32(np.finfo(np.float32).tiny)
 
-# the benchmark spec tolerances
+# parity tolerances: reduced sums, fp32 state, bf16 parameters, norm
 RTOL_REDUCED = 1e-6
 RTOL_STATE = 1e-5
 BF16_ULP = 1
