@@ -267,6 +267,7 @@ class Workload:
         self.params_per_step = (min(max(cfg["psi"] - owner * self.S, 0), self.S)
                                 if owner >= 0 else cfg["psi"])
         self.nb = self.lp.n_buckets
+        self._make_chunks()
 
     def make_graph(self):
         """The step captured as CUDA graphs (zero_partitioned_optimizer_step_b200.graph)."""
@@ -284,6 +285,7 @@ class Workload:
         self.lp = self.Z.zero_plan(cfg["psi"], cfg["nd"], cfg["stage"], bucket_elems,
                                    unit_elems=cfg["units"])
         self.nb = self.lp.n_buckets
+        self._make_chunks()
 
     def bucket_elems(self, b):
         """Elements bucket b processes (the owner's part in the owner view)."""
@@ -305,16 +307,28 @@ class Workload:
         if events is None:
             Z.zero_step(self.lp, self.G, self.w, self.m, self.v, self.params, self.adam, t, **kw)
         else:
-            for b in range(self.nb):
-                events[b].record(stream)
+            for i, (lo, hi, _) in enumerate(self.chunks):
+                events[i].record(stream)
                 Z.zero_step_buckets(self.lp, self.G, self.w, self.m, self.v, self.params,
-                                    self.adam, t, b, 1, **kw)
-            events[self.nb].record(stream)
+                                    self.adam, t, lo, hi - lo, **kw)
+            events[len(self.chunks)].record(stream)
         if self.layer is not None:
             n_units = len(self.units)
             for u in list(range(n_units)) + list(reversed(range(n_units))):
                 Z.zero_gather_layer(self.lp, u, self.params, self.layer[:self.units[u][0]], stream)
                 Z.zero_release_layer(self.lp, u)
+
+    def _make_chunks(self):
+        """Bucket ranges that each hold exactly one bucket with work for this
+        view (the one-owner view skips the buckets its shard is not in), so a
+        call per range launches one bucket kernel: [(first, end, elems)]."""
+        act = [b for b in range(self.nb) if self.bucket_elems(b) > 0]
+        out, lo = [], 0
+        for i, b in enumerate(act):
+            hi = b + 1 if i < len(act) - 1 else self.nb
+            out.append((lo, hi, self.bucket_elems(b)))
+            lo = hi
+        self.chunks = out
 
     def launches_per_step(self):
         n = sum(1 for b in range(self.nb) if self.bucket_elems(b) > 0)
@@ -409,7 +423,7 @@ def run_ours(args, cfg, rank, world, dist):
     torch.cuda.synchronize()
 
     n_ev = args.steps if sg is None else min(args.steps, 50)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(wl.nb + 1)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.chunks) + 1)]
               for _ in range(n_ev)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -440,11 +454,9 @@ def run_ours(args, cfg, rank, world, dist):
     k1_time = 0.0
     k1_elems = 0
     for k in range(n_ev):
-        for b in range(wl.nb):
-            if wl.bucket_elems(b) == 0:
-                continue
-            k1_time += events[k][b].elapsed_time(events[k][b + 1]) / 1e3
-            k1_elems += wl.bucket_elems(b)
+        for i, (_, _, n) in enumerate(wl.chunks):
+            k1_time += events[k][i].elapsed_time(events[k][i + 1]) / 1e3
+            k1_elems += n
     elapsed = max_over_ranks(elapsed, dist, dev)
 
     # end to end through the public API: gradients from pinned host memory
@@ -490,7 +502,7 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=Non
     per_elem = wl.step_bytes / wl.elems
     k1_bytes = per_elem * k1_elems
     achieved = k1_bytes / k1_time / 1e9
-    n_launch = (n_ev or args.steps) * sum(1 for b in range(wl.nb) if wl.bucket_elems(b) > 0)
+    n_launch = (n_ev or args.steps) * len(wl.chunks)
     tr = (k1_traffic_per_elem() if (args.config == "gpt2_small" and args.psi is None
                                     and wl.Z.zero_step_kernel(wl.lp, wl.owner) == "k_step_tma") else None)
     kname = wl.Z.zero_step_kernel(wl.lp, wl.owner)
@@ -550,14 +562,14 @@ def run_sweep(args, rank, world, dist):
                 torch.cuda.synchronize()
                 elapsed = s0.elapsed_time(s1) / 1e3
                 # again with an event around every bucket, for the kernel's own rate
-                events = [[torch.cuda.Event(enable_timing=True) for _ in range(wl.nb + 1)]
+                events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.chunks) + 1)]
                           for _ in range(args.steps)]
                 for k in range(args.steps):
                     wl.step(args.warmup + args.steps + 1 + k, stream, events[k])
                 torch.cuda.synchronize()
-                k1_time = sum(events[k][b].elapsed_time(events[k][b + 1]) / 1e3
-                              for k in range(args.steps) for b in range(wl.nb))
-                k1_elems = args.steps * sum(wl.bucket_elems(b) for b in range(wl.nb))
+                k1_time = sum(events[k][i].elapsed_time(events[k][i + 1]) / 1e3
+                              for k in range(args.steps) for i in range(len(wl.chunks)))
+                k1_elems = args.steps * sum(n for _, _, n in wl.chunks)
                 a = argparse.Namespace(**vars(args))
                 a.config = "sweep"
                 a.no_cpu_baseline = True

@@ -66,6 +66,18 @@ __device__ __forceinline__ bool not_finite(float x) {
     return (__float_as_uint(x) & 0x7f800000u) == 0x7f800000u;
 }
 
+// Programmatic dependent launch.  A bucket kernel lets the next one in the
+// stream launch as soon as it starts, so that the next bucket's CTAs take
+// each SM as this one's drain from it; the only memory consecutive bucket
+// kernels share is the norm slots, so each waits for its predecessor to
+// complete before adding to them.  Every CTA waits before it exits, so a
+// kernel never completes before its predecessor.  Both are no-ops without
+// the launch attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // The Adam constants of a launch: from device memory when the caller
 // supplied them there (so that a captured graph can be replayed for a new t),
 // else the launch arguments.

@@ -60,6 +60,7 @@ using namespace zero_dev;
 // per SM the register budget is sized for.
 template <bool OWNER_MAP, int RB, int MINB>
 __global__ void __launch_bounds__(kThreads, MINB) k_step_vec8(const StepArgs a) {
+    pdl_launch_dependents();
     const AdamConsts C = consts_of(a);
     const uint64_t nvec = (a.j1 - a.j0) >> 3;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kThreads, MINB) k_step_vec8(const StepArgs a) 
         for (uint32_t r = 0; r < a.n_prow; ++r)
             __stcs(reinterpret_cast<uint4 *>(p + uint64_t(r) * a.param_stride), pk);
     }
+    pdl_wait();
     if (a.ws_mode) block_partials(acc, bad, a);
 }
 
@@ -427,6 +429,39 @@ zero_status_t check_launch(const char *what) {
 
 bool mult8(int64_t x) { return (uint64_t(x) & 7u) == 0; }
 
+// Launch with or without programmatic dependent launch on the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_ex(void (*kernel)(Params...), uint32_t grid, uint32_t block, size_t smem,
+                      cudaStream_t stream, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// ZERO_PDL=0 turns programmatic dependent launch off (for comparison).
+bool pdl_enabled() {
+    const char *s = std::getenv("ZERO_PDL");
+    return !(s && s[0] == '0');
+}
+
+// Gradient rows a thread of the 16-byte-load kernel keeps in flight: 8 for
+// more than 16 ranks (read-heavy), else 4.  ZERO_LDG_RB=4|8 overrides.
+int ldg_rows(uint32_t nd) {
+    if (const char *e = std::getenv("ZERO_LDG_RB")) {
+        if (std::strcmp(e, "8") == 0) return 8;
+        if (std::strcmp(e, "4") == 0) return 4;
+    }
+    return nd > 16 ? 8 : 4;
+}
+
 struct Launcher {
     DeviceShapes shapes;
     cudaStream_t stream;
@@ -434,6 +469,7 @@ struct Launcher {
     bool use_tma = false;
     zero_tma::Ring ring{};
     uint32_t launches = 0;
+    bool pdl = true;  // vector-kernel launches after the first may overlap their predecessor
 
     zero_status_t run(StepArgs a, bool owner_map, bool vec_ok) {
         if (a.j0 >= a.j1) return ZERO_OK;
@@ -443,18 +479,19 @@ struct Launcher {
             b.j0 = j0;
             b.j1 = j1;
             b.ws_mode = want_ws ? 1 : 0;
+            const bool dep = pdl && launches > 0;
             if (vec && use_tma) {
                 const uint64_t tiles = (j1 - j0 + ring.tile - 1) / ring.tile;
                 const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
                 const size_t smem = size_t(ring.stages) * ring.stage_bytes;
                 TmaKernel f = owner_map ? tma_kernel<true>(ring.groups, ring.vw)
                                         : tma_kernel<false>(ring.groups, ring.vw);
-                f<<<grid, zero_tma::kThreads, smem, stream>>>(b, ring);
+                launch_ex(f, grid, zero_tma::kThreads, smem, stream, dep, b, ring);
             } else if (vec) {
-                if (owner_map)
-                    k_step_vec8<true, kRB, kMinB><<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
-                else
-                    k_step_vec8<false, kRB, kMinB><<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
+                const bool rb8 = ldg_rows(b.nd) == 8;
+                auto f = owner_map ? (rb8 ? k_step_vec8<true, 8, kMinB> : k_step_vec8<true, kRB, kMinB>)
+                                   : (rb8 ? k_step_vec8<false, 8, kMinB> : k_step_vec8<false, kRB, kMinB>);
+                launch_ex(f, shapes.grid_ldg, kThreads, 0, stream, dep, b);
             } else {
                 k_step_scalar<<<shapes.grid_ldg, kThreads, 0, stream>>>(b);
             }
@@ -601,6 +638,7 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     L.shapes = shapes;
     L.stream = static_cast<cudaStream_t>(stream_);
     L.want_ws = b->grad_norm_sq || b->overflow;
+    L.pdl = pdl_enabled();
     const int choice = kernel_choice();
     L.use_tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, &L.ring)
                             : choice != 1 && choose_ring(p->nd, a.n_prow == 1, shapes.tma_smem, &L.ring);

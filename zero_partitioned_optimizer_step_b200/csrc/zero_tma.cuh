@@ -245,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
     const uint32_t NS = ring.stages;
     const uint64_t n_tiles = (a.j1 - a.j0 + T - 1) / T;
 
+    zero_dev::pdl_launch_dependents();
     if (threadIdx.x == 0) {
         for (uint32_t s = 0; s < NS; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -366,6 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
         if (gt == 0) mbar_arrive(&empty_bar[s]);
     }
 
+    zero_dev::pdl_wait();  // predecessor done: its norm slots are final
     if (a.ws_mode) {
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
