@@ -78,6 +78,10 @@ def parse_args():
                     help="one-owner workloads: owner shard size (psi = nd * shard)")
     ap.add_argument("--layers", type=int, default=None,
                     help="stage-3 layer-wise workload: number of transformer blocks")
+    ap.add_argument("--peer", action="store_true",
+                    help="time the ranks-as-devices step (zero_step_peers): on one GPU the Nd "
+                         "ranks as separate allocations; under torchrun Nd = N GPUs, peers "
+                         "mapped through CUDA IPC")
     return ap.parse_args()
 
 
@@ -536,6 +540,159 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=Non
     return out
 
 
+NVLINK_GBS = 770.0   # measured peer copy per direction per GPU on this kind of node
+
+
+def run_peer(args, cfg, rank, world, dist):
+    """--peer: the ranks-as-devices step.  Each rank's buffers are its own
+    allocations: its bf16 gradient [psi_pad], its bf16 replica [psi_pad]
+    (stage 3: its shard [S]) and its fp32 shard of w, m, v.  On one GPU the
+    workload's Nd ranks all live on it and a step is Nd calls of
+    zero_step_peers, one per rank (the kernel then runs at HBM speed).  Under
+    torchrun Nd = N and every rank is one GPU: PeerStep maps the peers'
+    buffers through CUDA IPC, and the step's reduce-scatter and all-gather
+    are the kernel's NVLink loads and stores."""
+    import torch
+    import zero_partitioned_optimizer_step_b200 as Z
+    from zero_partitioned_optimizer_step_b200 import inputs
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    if cfg["owner_view"] >= 0:
+        raise SystemExit("--peer: the one-owner view has no counterpart; pick an all-ranks workload")
+    if cfg["stage"] == 0:
+        raise SystemExit("--peer: stage 0 keeps the full state on every rank")
+    if args.graph:
+        raise SystemExit("--peer: --graph is not supported")
+    nd = world if world > 1 else cfg["nd"]
+    lp = Z.zero_plan(cfg["psi"], nd, cfg["stage"], cfg["bucket_elems"], unit_elems=cfg["units"])
+    units = lp.units()
+    unit_len, unit_pad = [u[0] for u in units], [u[1] for u in units]
+    S, psi_pad = lp.S, lp.psi_pad
+    adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
+    w_log = inputs.master_logical(unit_len, unit_pad, cfg["seed_id"], dev)
+    ranks = range(nd) if world == 1 else [rank]
+    R = {}
+    for r in ranks:
+        g = torch.empty(psi_pad, dtype=torch.bfloat16, device=dev)
+        inputs.grad_row(g, unit_len, unit_pad, cfg["sigma"], inputs.seed_for(cfg["seed_id"], r, 1),
+                        cfg["outlier_frac"])
+        w = torch.cat([w_log[U + r * s:U + (r + 1) * s] for (_, _, s, U, _) in units])
+        n_p = psi_pad if cfg["stage"] <= 2 else S
+        R[r] = dict(g=g, w=w, m=torch.zeros(S, dtype=torch.float32, device=dev),
+                    v=torch.zeros(S, dtype=torch.float32, device=dev),
+                    p=torch.empty(n_p, dtype=torch.bfloat16, device=dev),
+                    norm=torch.zeros(1, dtype=torch.float64, device=dev),
+                    ovf=torch.zeros(1, dtype=torch.int32, device=dev), ws=Z.workspace_for(lp, dev))
+    del w_log
+    ps = None
+    if world > 1:
+        from zero_partitioned_optimizer_step_b200.peer import PeerStep
+        b = R[rank]
+        ps = PeerStep(lp, b["g"], b["p"], b["w"], b["m"], b["v"])
+    grads = [R[q]["g"] for q in range(nd)] if world == 1 else None
+    params = [R[q]["p"] for q in range(nd)] if world == 1 else None
+
+    def one_step(t, ev=None):
+        if ps is not None:
+            b = R[rank]
+            ps.step(adam, t, grad_norm_sq=b["norm"], overflow=b["ovf"], workspace=b["ws"], events=ev)
+            return
+        if ev is not None:
+            ev[0].record()
+        for r in ranks:
+            b = R[r]
+            Z.zero_step_peers(lp, r, grads, params, b["w"], b["m"], b["v"], adam, t,
+                              grad_norm_sq=b["norm"], overflow=b["ovf"], workspace=b["ws"])
+        if ev is not None:
+            ev[1].record()
+
+    t = 1
+    for _ in range(args.warmup):
+        one_step(t)
+        t += 1
+    Z.zero_stream_status()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index).start()
+    time.sleep(0.2)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for k in range(args.steps):
+        one_step(t + k, events[k])
+    end.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    Z.zero_stream_status()
+    elapsed = max_over_ranks(start.elapsed_time(end) / 1e3, dist, dev)
+    k_time = max_over_ranks(sum(a.elapsed_time(b) for a, b in events) / 1e3, dist, dev)
+    if ps is not None:
+        ps.close()
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    hbm_step = Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_STEP)
+    if world == 1:
+        per_launch_bytes = hbm_step / max(1, nd)
+        roof = {"kernel": "k_step_peer (rank r's reduce-scatter + Adam + all-gather over its "
+                          "ranks' buffers; %d calls per step)" % nd,
+                "bound": "hbm", "achieved": hbm_step * args.steps / k_time / 1e9, "peak": peak,
+                "unit": "GB/s", "peak_kind": peak_kind + " (copy bandwidth)", "traffic": None,
+                "algorithmic_bytes_per_call": per_launch_bytes,
+                "avg_call_ms": k_time / args.steps / nd * 1e3}
+    else:
+        # per direction: 2(Nd-1)S bytes of peer gradient reads come in and (stages
+        # 1-2) as many bytes of replica stores go out; stage-3 stores stay local
+        link = 2 * (nd - 1) * S
+        roof = {"kernel": "k_step_peer (one rank per GPU, peer loads and stores over NVLink)",
+                "bound": "nvlink", "achieved": link * args.steps / k_time / 1e9, "peak": NVLINK_GBS,
+                "unit": "GB/s", "peak_kind": "measured peer copy per direction", "traffic": None,
+                "algorithmic_nvlink_bytes_per_direction": link}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return {
+        "metric": METRIC, "value": cfg["psi"] * args.steps / elapsed / 1e9, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg["workload"] + ", ranks as devices (zero_step_peers)",
+                   "psi": cfg["psi"], "nd": nd, "stage": cfg["stage"],
+                   "bucket_elems": cfg["bucket_elems"], "peer": True,
+                   "hbm_bytes_per_step": hbm_step,
+                   "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (hbm_step / 1e9)},
+        "roofline": roof, "e2e": None,
+        "gpu_launches": sum(peer_launches(lp, r) for r in ranks) * args.steps, "clocks": clk,
+    }
+
+
+def peer_launches(lp, r):
+    """Kernels zero_step_peers launches for rank r in one step with the norm
+    on: per bucket, r's part split into an unaligned head, an 8-aligned body
+    and a tail (all scalar when r's storage offset is not a multiple of 8),
+    then the finalize."""
+    import zero_partitioned_optimizer_step_b200 as Z
+    units = lp.units()
+    n = 0
+    for b in range(lp.n_buckets):
+        u = lp.query(Z.ZERO_Q_BUCKET_UNIT, b)
+        lo_b, hi_b = lp.query(Z.ZERO_Q_BUCKET_BEGIN, b), lp.query(Z.ZERO_Q_BUCKET_END, b)
+        _, _, s, U, O = units[u]
+        lo = U + r * s
+        p0, p1 = max(lo_b, lo), min(hi_b, lo + s)
+        if p0 >= p1:
+            continue
+        vlo, vhi = (p0 + 7) // 8 * 8, p1 // 8 * 8
+        if (O - lo) % 8 or vlo >= vhi:
+            n += 1
+        else:
+            n += (p0 < vlo) + 1 + (vhi < p1)
+    return n + 1
+
+
 def run_sweep(args, rank, world, dist):
     """The bucket-size sweep (5e8 params): for each Nd one set of buffers, then
     every bucket size from 1 MB to 512 MB of one rank's bf16 gradient."""
@@ -623,7 +780,7 @@ def main():
         if args.sweep:
             run_sweep(args, rank, world, dist)
             return 0
-        res = run_ours(args, cfg, rank, world, dist)
+        res = (run_peer if args.peer else run_ours)(args, cfg, rank, world, dist)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

@@ -73,7 +73,7 @@
 extern "C" {
 #endif
 
-#define ZERO_ABI_VERSION 2
+#define ZERO_ABI_VERSION 3
 
 typedef enum zero_status {
     ZERO_OK = 0,
@@ -324,6 +324,122 @@ zero_status_t zero_gather_layer(zero_plan_t *plan, uint32_t unit,
  * layers form memory peaks).  Host only.  ZERO_EINVAL: unit out of range.
  * ZERO_ESTATE: the unit is not live. */
 zero_status_t zero_release_layer(zero_plan_t *plan, uint32_t unit);
+
+/* ---------------------------------------------------------------------------
+ * Ranks as devices.  The calls above hold all Nd ranks on one GPU.  The calls
+ * below run one rank's share of the same step when each rank has its own
+ * buffers, which is how ZeRO runs: rank r's process calls them on its own
+ * GPU, and every other rank's gradient and parameter replica are reachable
+ * from that GPU through plain device pointers.  On one node those are peer
+ * mappings over NVLink/NVSwitch (zero_ipc_open() of another process's
+ * buffer); the same calls also accept local buffers, so that Nd ranks can be
+ * separate allocations on one GPU.
+ *
+ * Rank r's step, per bucket (stages 1-3; [MM] section "但 GPU 只存四分之一…":
+ * each rank sends the gradient of a shard to the rank that owns it, which
+ * updates it; the updated parameters are then exchanged):
+ *   reduce-scatter: for every element p that r owns, read G_q[p] from every
+ *     rank q directly from q's memory and add them in rank order 0..Nd-1
+ *     from rank 0's value, in fp32 (the same sum as zero_step);
+ *   owner Adam on r's fp32 state, which is local;
+ *   all-gather: store bf16(w) straight into every rank's replica (stages 1-2)
+ *     or into r's own parameter shard (stage 3).
+ * The collective is inside the kernel: there is no separate reduce-scatter
+ * or all-gather.  Every rank's results are bit-identical to zero_step's on
+ * the same inputs.  Each element is read and written by exactly one rank (its
+ * owner), so the ranks' kernels never wait for one another and share no
+ * flags.  The caller orders the step against the other ranks: all ranks'
+ * gradients must be complete before any rank's call runs, and no rank may
+ * read its replica or overwrite a gradient until every rank's call has
+ * finished (e.g. a one-element all-reduce on the stream before and after;
+ * the kernels end with a system-scope fence so that their stores to peers
+ * are performed when they complete).  Stage 0 keeps a full state on every
+ * rank, which this layout does not describe: ZERO_EINVAL.
+ * ------------------------------------------------------------------------- */
+#define ZERO_MAX_PEERS 128u
+
+typedef struct zero_peer_bufs {
+    uint32_t rank;           /* r: the owner whose shard this call updates */
+    uint32_t reserved;       /* 0 */
+    const void *const *grads;/* HOST array [Nd] of device pointers: grads[q] =
+                                rank q's bf16 gradient [psi_pad] in logical
+                                order (padding zero), readable from this
+                                device; 16-byte aligned */
+    void *const *params;     /* HOST array [Nd].  Stages 1-2: params[q] = rank
+                                q's bf16 replica [psi_pad], logical order,
+                                writable from this device.  Stage 3: only
+                                params[rank] is used: r's bf16 owner shard [S]
+                                in storage order */
+    float *master;           /* r's fp32 master shard [S], storage order; in/out */
+    float *exp_avg;          /* r's fp32 m [S]; in/out */
+    float *exp_avg_sq;       /* r's fp32 v [S]; in/out */
+    float *reduced_grad;     /* optional fp32 [S] out: r's g_sum */
+    double *grad_norm_sq;    /* optional device scalar out: sum of g_sum^2 over
+                                r's shard (sum it over ranks for the global
+                                norm) */
+    int32_t *overflow;       /* optional device scalar out: 1 if a g_sum of
+                                r's shard is inf or NaN */
+    void *workspace;         /* needed iff grad_norm_sq or overflow is set */
+    uint64_t workspace_bytes;
+    const void *adam_consts; /* optional, as in zero_bufs_t */
+} zero_peer_bufs_t;
+
+/* Rank bufs->rank's part of buckets [first_bucket, first_bucket + n_buckets)
+ * of a step (n_buckets = zero_plan_query(ZERO_Q_N_BUCKETS) for the whole
+ * step), as described above; the norm workspace is reset by the call that
+ * contains bucket 0 and reported by the call that contains the last.  The
+ * grads and params arrays are read on the host during the call only.  Bytes
+ * per owned element: 2Nd read from the ranks' gradients (2(Nd-1) of them
+ * from peers), 12 read + 12 written of local state, 2Nd written to replicas
+ * (2(Nd-1) to peers), or 2 at stage 3.  ZERO_EINVAL: as zero_step, or stage
+ * 0, Nd > ZERO_MAX_PEERS, rank out of range, a NULL or misaligned entry of
+ * grads or params.  ZERO_ECUDA: launch failure. */
+zero_status_t zero_step_peers(const zero_plan_t *plan, const zero_peer_bufs_t *bufs,
+                              const zero_adam_t *adam, uint64_t t, uint64_t first_bucket,
+                              uint64_t n_buckets, void *stream);
+
+/* Stage 3 with ranks as devices: materialise unit `unit` into full_layer
+ * [len_u] by reading owner q's slice from owner_params[q] (a HOST array [Nd]
+ * of device pointers to each rank's bf16 owner shard [S], readable from this
+ * device), in rank order.  Liveness as zero_gather_layer (the plan counts
+ * this rank's live units).  Errors as zero_gather_layer, plus ZERO_EINVAL
+ * for a NULL or misaligned entry of owner_params. */
+zero_status_t zero_gather_layer_peers(zero_plan_t *plan, uint32_t unit,
+                                      const void *const *owner_params, void *full_layer,
+                                      void *stream);
+
+/* Sharing a buffer with another process on the same node (CUDA IPC).  The
+ * handle names the buffer's whole allocation plus the buffer's offset in it,
+ * so buffers carved out of a larger allocation (a caching allocator's) can be
+ * shared; the allocation must come from cudaMalloc (not from a virtual-memory
+ * or managed allocator).  A handle is plain bytes: send it to the other ranks
+ * by any means. */
+typedef struct zero_ipc_handle {
+    unsigned char handle[64];/* cudaIpcMemHandle_t of the allocation */
+    uint64_t offset;         /* buffer start - allocation start, bytes */
+    uint64_t alloc_bytes;    /* size of the allocation */
+    uint64_t exporter_va;    /* allocation start in the exporting process */
+    int32_t device;          /* CUDA ordinal of the buffer in the exporter */
+    int32_t exporter_pid;    /* process that exported it */
+} zero_ipc_handle_t;
+
+/* Describe the device buffer at ptr for zero_ipc_open() in another process.
+ * ZERO_EINVAL: NULL, or ptr is not device memory from cudaMalloc.
+ * ZERO_ECUDA: the CUDA call failed. */
+zero_status_t zero_ipc_export(const void *ptr, zero_ipc_handle_t *out);
+
+/* Map a buffer exported by zero_ipc_export() into this process on the current
+ * CUDA device (peer access is enabled as needed) and return its address.  A
+ * handle exported by this same process returns the original address without
+ * a mapping.  Opening several buffers of one allocation maps it once
+ * (reference-counted).  ZERO_EINVAL: NULL.  ZERO_ECUDA: the mapping failed
+ * (no peer access between the two devices, or the exporter has freed it). */
+zero_status_t zero_ipc_open(const zero_ipc_handle_t *h, void **ptr);
+
+/* Undo one zero_ipc_open(); the mapping goes when its last buffer is closed.
+ * ZERO_EINVAL: ptr was not returned by zero_ipc_open() (or already closed).
+ * ZERO_ECUDA: unmapping failed. */
+zero_status_t zero_ipc_close(void *ptr);
 
 typedef enum zero_bytes_kind {
     ZERO_BYTES_COMM_ELEMS_PER_RANK = 0, /* ring model, elements one rank sends

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_function():
     assert len(names) >= 11
     for n in names:
         assert hasattr(L, n), n
-    assert L.zero_abi_version() == 2
+    assert L.zero_abi_version() == 3
 
 
 def test_status_strings():

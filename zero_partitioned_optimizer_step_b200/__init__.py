@@ -71,6 +71,25 @@ class _Bufs(ctypes.Structure):
                 ("owner_view", ctypes.c_int32), ("adam_consts", ctypes.c_void_p)]
 
 
+class _PeerBufs(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+                ("grads", ctypes.POINTER(ctypes.c_void_p)), ("params", ctypes.POINTER(ctypes.c_void_p)),
+                ("master", ctypes.c_void_p), ("exp_avg", ctypes.c_void_p),
+                ("exp_avg_sq", ctypes.c_void_p), ("reduced_grad", ctypes.c_void_p),
+                ("grad_norm_sq", ctypes.c_void_p), ("overflow", ctypes.c_void_p),
+                ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_uint64),
+                ("adam_consts", ctypes.c_void_p)]
+
+
+class _IpcHandle(ctypes.Structure):
+    _fields_ = [("handle", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64),
+                ("alloc_bytes", ctypes.c_uint64), ("exporter_va", ctypes.c_uint64),
+                ("device", ctypes.c_int32), ("exporter_pid", ctypes.c_int32)]
+
+
+ZERO_MAX_PEERS = 128
+IPC_HANDLE_BYTES = ctypes.sizeof(_IpcHandle)
+
 _LIB = None
 
 
@@ -116,6 +135,17 @@ def lib():
         L.zero_adam_consts.argtypes = [ctypes.POINTER(_Adam), u64, vp]
         L.zero_stream_status.restype = st
         L.zero_stream_status.argtypes = [vp]
+        L.zero_step_peers.restype = st
+        L.zero_step_peers.argtypes = [vp, ctypes.POINTER(_PeerBufs), ctypes.POINTER(_Adam),
+                                      u64, u64, u64, vp]
+        L.zero_gather_layer_peers.restype = st
+        L.zero_gather_layer_peers.argtypes = [vp, ctypes.c_uint32, ctypes.POINTER(vp), vp, vp]
+        L.zero_ipc_export.restype = st
+        L.zero_ipc_export.argtypes = [vp, ctypes.POINTER(_IpcHandle)]
+        L.zero_ipc_open.restype = st
+        L.zero_ipc_open.argtypes = [ctypes.POINTER(_IpcHandle), ctypes.POINTER(vp)]
+        L.zero_ipc_close.restype = st
+        L.zero_ipc_close.argtypes = [vp]
         L.zero_status_str.restype = ctypes.c_char_p
         L.zero_status_str.argtypes = [ctypes.c_int]
         L.zero_last_error.restype = ctypes.c_char_p
@@ -384,3 +414,91 @@ def workspace_for(plan, device="cuda"):
     """A caller-owned device workspace of the size the norm/overflow needs."""
     import torch
     return torch.empty(plan.query(ZERO_Q_WORKSPACE_BYTES), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------ ranks as devices
+def _dev_ptr(x, dtype, name):
+    """A device pointer from a CUDA tensor or an int address (a peer mapping
+    from zero_ipc_open); None -> NULL."""
+    if x is None or isinstance(x, int):
+        return x
+    return _ptr(x, dtype, name)
+
+
+def _ptr_array(items, dtype, name):
+    arr = (ctypes.c_void_p * len(items))()
+    for q, x in enumerate(items):
+        arr[q] = _dev_ptr(x, dtype, "%s[%d]" % (name, q))
+    return arr
+
+
+def zero_step_peers(plan, rank, grads, params, master, exp_avg, exp_avg_sq, adam, t,
+                    first_bucket=0, n_buckets=None, stream=None, reduced_grad=None,
+                    grad_norm_sq=None, overflow=None, workspace=None, adam_consts=None):
+    """Rank `rank`'s part of a step whose ranks have their own buffers.
+
+    grads: Nd bf16 gradients [psi_pad] (CUDA tensors, or int addresses of peer
+    mappings), one per rank.  params: Nd bf16 replicas [psi_pad] at stages
+    1-2; at stage 3 only params[rank] (this rank's owner shard [S]) is used.
+    master / exp_avg / exp_avg_sq: this rank's fp32 shard [S].
+    """
+    import torch
+    nd = plan.nd
+    if len(grads) != nd or len(params) != nd:
+        raise ValueError("grads and params must hold one entry per rank (%d)" % nd)
+    g_arr = _ptr_array(grads, torch.bfloat16, "grads")
+    p_arr = _ptr_array(params, torch.bfloat16, "params")
+    b = _PeerBufs()
+    b.rank = int(rank)
+    b.grads = ctypes.cast(g_arr, ctypes.POINTER(ctypes.c_void_p))
+    b.params = ctypes.cast(p_arr, ctypes.POINTER(ctypes.c_void_p))
+    b.master = _ptr(master, torch.float32, "master")
+    b.exp_avg = _ptr(exp_avg, torch.float32, "exp_avg")
+    b.exp_avg_sq = _ptr(exp_avg_sq, torch.float32, "exp_avg_sq")
+    b.reduced_grad = _ptr(reduced_grad, torch.float32, "reduced_grad")
+    b.grad_norm_sq = _ptr(grad_norm_sq, torch.float64, "grad_norm_sq")
+    b.overflow = _ptr(overflow, torch.int32, "overflow")
+    b.workspace = _ptr(workspace, None, "workspace")
+    b.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    b.adam_consts = _ptr(adam_consts, torch.float32, "adam_consts")
+    n = plan.n_buckets - int(first_bucket) if n_buckets is None else int(n_buckets)
+    _check(lib().zero_step_peers(plan.handle, ctypes.byref(b), ctypes.byref(make_adam(adam)),
+                                 int(t), int(first_bucket), n, _stream(stream)))
+
+
+def zero_gather_layer_peers(plan, unit, owner_params, full_layer, stream=None):
+    """Stage 3: materialise unit `unit` from the Nd owners' bf16 shards
+    (tensors or int addresses of peer mappings), in rank order."""
+    import torch
+    if len(owner_params) != plan.nd:
+        raise ValueError("owner_params must hold one entry per rank (%d)" % plan.nd)
+    arr = _ptr_array(owner_params, torch.bfloat16, "owner_params")
+    _check(lib().zero_gather_layer_peers(plan.handle, int(unit),
+                                         ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)),
+                                         _ptr(full_layer, torch.bfloat16, "full_layer"),
+                                         _stream(stream)))
+
+
+def zero_ipc_export(tensor_or_ptr):
+    """IPC handle (bytes, IPC_HANDLE_BYTES long) of a CUDA buffer, to send to
+    another process on the node."""
+    h = _IpcHandle()
+    p = tensor_or_ptr if isinstance(tensor_or_ptr, int) else _ptr(tensor_or_ptr, None, "buffer")
+    _check(lib().zero_ipc_export(ctypes.c_void_p(p), ctypes.byref(h)))
+    return bytes(h)
+
+
+def zero_ipc_open(handle):
+    """Map a buffer exported by another process (bytes from zero_ipc_export)
+    on the current CUDA device; returns its address as an int."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is %d bytes" % IPC_HANDLE_BYTES)
+    h = _IpcHandle.from_buffer_copy(handle)
+    out = ctypes.c_void_p()
+    _check(lib().zero_ipc_open(ctypes.byref(h), ctypes.byref(out)))
+    return int(out.value)
+
+
+def zero_ipc_close(ptr):
+    """Undo one zero_ipc_open()."""
+    _check(lib().zero_ipc_close(ctypes.c_void_p(int(ptr))))

@@ -109,7 +109,7 @@ __device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w
 // Per-CTA partials of the gradient-norm / overflow reduction, added to slot
 // blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
 // so the reported norm is the same on every run of the same launch shapes.
-__device__ __forceinline__ void block_partials(double acc, uint32_t bad, const StepArgs &a) {
+__device__ __forceinline__ void block_partials(double acc, uint32_t bad, double *ws_norm, uint32_t *ws_bad) {
     __shared__ double sd[kThreads / 32];
     __shared__ uint32_t sb[kThreads / 32];
 #pragma unroll
@@ -130,8 +130,41 @@ __device__ __forceinline__ void block_partials(double acc, uint32_t bad, const S
             t += sd[i];
             b += sb[i];
         }
-        a.ws_norm[blockIdx.x] += t;
-        a.ws_bad[blockIdx.x] = min(a.ws_bad[blockIdx.x] + b, 0x7fffffffu);
+        ws_norm[blockIdx.x] += t;
+        ws_bad[blockIdx.x] = min(ws_bad[blockIdx.x] + b, 0x7fffffffu);
+    }
+}
+
+__device__ __forceinline__ void block_partials(double acc, uint32_t bad, const StepArgs &a) {
+    block_partials(acc, bad, a.ws_norm, a.ws_bad);
+}
+
+// K3: fixed-order sum of the per-CTA partials of one step (one block).  Each
+// translation unit that includes this header has its own copy (static).
+static __global__ void __launch_bounds__(kThreads) k_finalize(const double *ws_norm, const uint32_t *ws_bad,
+                                                      uint32_t slots, double *norm_out,
+                                                      int32_t *overflow_out) {
+    __shared__ double sd[kThreads];
+    __shared__ uint32_t sb[kThreads];
+    double t = 0.0;
+    uint32_t b = 0;
+    for (uint32_t i = threadIdx.x; i < slots; i += kThreads) {
+        t += ws_norm[i];
+        b |= ws_bad[i] != 0;
+    }
+    sd[threadIdx.x] = t;
+    sb[threadIdx.x] = b;
+    __syncthreads();
+    for (int s = kThreads / 2; s > 0; s >>= 1) {
+        if (threadIdx.x < s) {
+            sd[threadIdx.x] += sd[threadIdx.x + s];
+            sb[threadIdx.x] |= sb[threadIdx.x + s];
+        }
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        if (norm_out) *norm_out = sd[0];
+        if (overflow_out) *overflow_out = sb[0] ? 1 : 0;
     }
 }
 

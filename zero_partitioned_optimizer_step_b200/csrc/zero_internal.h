@@ -44,6 +44,12 @@ struct BucketRange {
 };
 BucketRange bucket_range(const zero_plan_t &p, uint64_t b);
 
+// Stage-3 liveness of the gathers; the caller holds p.mu.  live_check
+// returns ZERO_ESTATE (message prefixed by `who`) if `unit` is live already
+// or max_live units are live; live_mark records a successful gather.
+zero_status_t live_check(const zero_plan_t &p, uint32_t unit, const char *who);
+void live_mark(zero_plan_t &p, uint32_t unit);
+
 // Workspace layout for the gradient-norm / overflow reduction: one fp64
 // partial and one u32 count per CTA slot, kMaxSlots slots, then 256 bytes
 // for the guarded step's decision (clip coefficient and skip flag).

@@ -273,6 +273,26 @@ ZERO_API zero_status_t zero_bytes_moved(const zero_plan_t *p, zero_bytes_kind_t 
     return set_error(ZERO_EINVAL, "zero_bytes_moved: unknown kind");
 }
 
+namespace zero_detail {
+
+zero_status_t live_check(const zero_plan_t &p, uint32_t unit, const char *who) {
+    if (p.live[unit])
+        return set_error(ZERO_ESTATE, std::string(who) + ": unit " + std::to_string(unit) + " is already live");
+    if (p.n_live >= p.max_live)
+        return set_error(ZERO_ESTATE, std::string(who) + ": max_live units are live; release one first");
+    return ZERO_OK;
+}
+
+void live_mark(zero_plan_t &p, uint32_t unit) {
+    p.live[unit] = 1;
+    p.n_live += 1;
+    p.live_bytes += 2 * p.unit_len[unit];
+    p.peak_live = std::max(p.peak_live, p.n_live);
+    p.peak_live_bytes = std::max(p.peak_live_bytes, p.live_bytes);
+}
+
+}  // namespace zero_detail
+
 ZERO_API zero_status_t zero_release_layer(zero_plan_t *p, uint32_t unit) {
     zero_detail::clear_error();
     if (!p) return set_error(ZERO_EINVAL, "zero_release_layer: NULL plan");

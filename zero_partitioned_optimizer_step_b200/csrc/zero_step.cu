@@ -192,34 +192,6 @@ __global__ void __launch_bounds__(kThreads) k_step_scalar(const StepArgs a) {
     if (a.ws_mode) block_partials(acc, bad, a);
 }
 
-// K3: fixed-order sum of the per-CTA partials of one step.
-__global__ void __launch_bounds__(kThreads) k_finalize(const double *ws_norm, const uint32_t *ws_bad,
-                                                      uint32_t slots, double *norm_out,
-                                                      int32_t *overflow_out) {
-    __shared__ double sd[kThreads];
-    __shared__ uint32_t sb[kThreads];
-    double t = 0.0;
-    uint32_t b = 0;
-    for (uint32_t i = threadIdx.x; i < slots; i += kThreads) {
-        t += ws_norm[i];
-        b |= ws_bad[i] != 0;
-    }
-    sd[threadIdx.x] = t;
-    sb[threadIdx.x] = b;
-    __syncthreads();
-    for (int s = kThreads / 2; s > 0; s >>= 1) {
-        if (threadIdx.x < s) {
-            sd[threadIdx.x] += sd[threadIdx.x + s];
-            sb[threadIdx.x] |= sb[threadIdx.x + s];
-        }
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        if (norm_out) *norm_out = sd[0];
-        if (overflow_out) *overflow_out = sb[0] ? 1 : 0;
-    }
-}
-
 // K2: full_layer[o*s_u + i] = owner_params[o*S + off_u + i] for the first
 // len_u elements; `cpo` CTAs per owner, owners in rank order.  Each thread
 // keeps four 16-byte loads in flight before it stores them.
@@ -684,16 +656,14 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
     if (!aligned16(owner_params) || !aligned16(full_layer))
         return set_error(ZERO_EINVAL, "zero_gather_layer: buffers must be 16-byte aligned");
     std::lock_guard<std::mutex> g(p->mu);
-    if (p->live[unit])
-        return set_error(ZERO_ESTATE, "zero_gather_layer: unit " + std::to_string(unit) + " is already live");
-    if (p->n_live >= p->max_live)
-        return set_error(ZERO_ESTATE, "zero_gather_layer: max_live units are live; release one first");
+    zero_status_t st = zero_detail::live_check(*p, unit, "zero_gather_layer");
+    if (st != ZERO_OK) return st;
     cudaError_t pre = cudaPeekAtLastError();
     if (pre != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_gather_layer: ") +
                                          cudaGetErrorString(pre));
     DeviceShapes shapes;
-    zero_status_t st = device_shapes(&shapes);
+    st = device_shapes(&shapes);
     if (st != ZERO_OK) return st;
     const uint64_t s_u = p->unit_shard[unit], off = p->unit_offset[unit], len = p->unit_len[unit];
     const int vec_ok = ((p->S | off | s_u) & 7u) == 0;
@@ -705,11 +675,7 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
         p->nd, cpo, vec_ok);
     st = check_launch("zero_gather_layer launch");
     if (st != ZERO_OK) return st;
-    p->live[unit] = 1;
-    p->n_live += 1;
-    p->live_bytes += 2 * len;
-    p->peak_live = std::max(p->peak_live, p->n_live);
-    p->peak_live_bytes = std::max(p->peak_live_bytes, p->live_bytes);
+    zero_detail::live_mark(*p, unit);
     return ZERO_OK;
 }
 
