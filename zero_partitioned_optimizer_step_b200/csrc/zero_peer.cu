@@ -28,8 +28,8 @@
 // traffic, not HBM, bounds it.  Ranks never wait for one another inside a
 // kernel (each element has one owner, so no two ranks touch the same bytes);
 // the caller orders whole steps across ranks on the host or with a stream
-// collective.  Each CTA ends with a system-scope fence, so its peer stores
-// are performed before the kernel counts as complete.
+// collective.  Each CTA ends with a system-scope fence after a CTA barrier,
+// so its peer stores are performed before the kernel counts as complete.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -79,6 +79,14 @@ struct PeerArgs {
 };
 
 __device__ __forceinline__ AdamConsts peer_consts(const PeerArgs &a) { return a.cdev ? *a.cdev : a.c; }
+
+// The CTA's stores (to peers included) are ordered before a system-scope
+// fence: the barrier makes every thread's stores precede thread 0's fence,
+// which is cumulative.  One fence per CTA instead of one per thread.
+__device__ __forceinline__ void cta_release_system() {
+    __syncthreads();
+    if (threadIdx.x == 0) __threadfence_system();
+}
 
 // K5, vector path: 8 elements per thread and iteration, kPeerRB gradient rows
 // loaded together (peer loads have a long latency) before their in-order
@@ -152,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, kPeerMinB) k_step_peer(const PeerArg
         pk.w = pack_bf16x2(wv[6], wv[7]);
         for (uint32_t q = 0; q < a.n_prow; ++q) __stcs(reinterpret_cast<uint4 *>(sp[q] + pi), pk);
     }
-    __threadfence_system();
+    cta_release_system();
     if (a.ws_mode) block_partials(acc, bad, a.ws_norm, a.ws_bad);
 }
 
@@ -188,7 +196,7 @@ __global__ void __launch_bounds__(kThreads) k_step_peer_scalar(const PeerArgs a,
         const uint16_t bits = *reinterpret_cast<uint16_t *>(&h);
         for (uint32_t q = 0; q < a.n_prow; ++q) sp[q][pi] = bits;
     }
-    __threadfence_system();
+    cta_release_system();
     if (a.ws_mode) block_partials(acc, bad, a.ws_norm, a.ws_bad);
 }
 
