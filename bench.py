@@ -4,14 +4,18 @@
                     [--config gpt2_small|toy|stage3_1p3b|owner_7p5b|sweep]
                     [--nd ND --bucket-mb MB]                 # one bucket-sweep point
                     [--sweep OUT.jsonl]                      # the whole bucket sweep
-                    [--graph]                                # replay the step as a CUDA graph
+                    [--eager]                                # launch every step from the host
 
 One step = the whole hot path over one batch of gradients: for every bucket,
 the fused reduce-scatter + owner Adam + all-gather kernel, then the
 gradient-norm / overflow reduction (stage 3 workloads add the forward and
-backward layer gathers).  The default workload is the GPT-2-small-shaped
-flat vector (124,439,808 parameters, Nd = 8 logical ranks, stage 2,
-25M-element buckets).  Inputs are resident in HBM when timing starts and one
+backward layer gathers).  The timed steps are replayed as a CUDA graph
+(graph.StepGraph: the same kernels, with the step's constants refreshed in
+device memory by a captured copy) unless the workload gathers layers or
+--eager is given; the dominant kernel's own rate is then taken from extra
+eager steps with an event around every bucket.  The default workload is the
+GPT-2-small-shaped flat vector (124,439,808 parameters, Nd = 8 logical
+ranks, stage 2, 25M-element buckets).  Inputs are resident in HBM when timing starts and one
 step touches ~7 GB, far more than the 126 MB L2, so no flush is needed.
 
 The metric is parameters updated per second (Gparams/s); the JSON line also
@@ -71,13 +75,28 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--graph", action="store_true",
-                    help="time the step replayed as a CUDA graph (workloads without layer gathers)")
+                    help="time the step replayed as a CUDA graph (the default where possible; "
+                         "for --sweep: add graph-replay numbers)")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the step launched from the host every time, not as a graph")
     ap.add_argument("--psi", type=int, default=None,
                     help="override the parameter count (flat single-unit workloads only)")
     ap.add_argument("--shard", type=int, default=None,
                     help="one-owner workloads: owner shard size (psi = nd * shard)")
     ap.add_argument("--layers", type=int, default=None,
                     help="stage-3 layer-wise workload: number of transformer blocks")
+    ap.add_argument("--guarded", action="store_true",
+                    help="time the two-pass guarded step (global-norm clip, skip on overflow)")
+    ap.add_argument("--max-grad-norm", type=float, default=1.0,
+                    help="--guarded: clip threshold (0 = no clipping)")
+    ap.add_argument("--prefetch", type=int, default=None,
+                    help="stage-3 workloads: gather the layers with a prefetch window of this "
+                         "depth on a side stream (default: one after the other)")
+    ap.add_argument("--weight-decay", type=float, default=0.0,
+                    help="decoupled weight decay (AdamW) of every step")
+    ap.add_argument("--reshard", type=int, default=None, metavar="ND2",
+                    help="time resharding the workload's owner-storage state (w, m, v; and the "
+                         "parameter shards at stage 3) from its Nd to ND2 ranks")
     ap.add_argument("--peer", action="store_true",
                     help="time the ranks-as-devices step (zero_step_peers): on one GPU the Nd "
                          "ranks as separate allocations; under torchrun Nd = N GPUs, peers "
@@ -220,7 +239,7 @@ def job_value(world, params_per_rank_step, steps, seconds):
 class Workload:
     """Device buffers of one configuration, built from the seeded generators."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, prefetch=None, weight_decay=0.0):
         import torch
         import zero_partitioned_optimizer_step_b200 as Z
         from zero_partitioned_optimizer_step_b200 import inputs
@@ -228,10 +247,13 @@ class Workload:
         self.cfg = cfg
         self.dev = device
         nd, stage, owner = cfg["nd"], cfg["stage"], cfg["owner_view"]
-        self.lp = Z.zero_plan(cfg["psi"], nd, stage, cfg["bucket_elems"], unit_elems=cfg["units"])
+        self.prefetch = prefetch
+        self.lp = Z.zero_plan(cfg["psi"], nd, stage, cfg["bucket_elems"], unit_elems=cfg["units"],
+                              max_live=1 + (prefetch or 0))
         self.units = self.lp.units()
         self.S, self.psi_pad = self.lp.S, self.lp.psi_pad
-        self.adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
+        self.adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd,
+                         weight_decay=weight_decay)
         unit_len = [u[0] for u in self.units]
         unit_pad = [u[1] for u in self.units]
         if owner >= 0:
@@ -262,6 +284,10 @@ class Workload:
         self.layer = None
         if stage == 3 and owner < 0:
             self.layer = torch.empty(max(unit_len), dtype=torch.bfloat16, device=device)
+            if prefetch:
+                self.ring = [self.layer] + [torch.empty(max(unit_len), dtype=torch.bfloat16, device=device)
+                                            for _ in range(prefetch)]
+                self.side = torch.cuda.Stream(device)
         self.owner = owner
         flags = Z.ZERO_BYTES_FLAG_OWNER_VIEW if owner >= 0 else 0
         self.step_bytes = Z.zero_bytes_moved(self.lp, Z.ZERO_BYTES_HBM_STEP, flags)
@@ -317,10 +343,24 @@ class Workload:
                                     self.adam, t, lo, hi - lo, **kw)
             events[len(self.chunks)].record(stream)
         if self.layer is not None:
-            n_units = len(self.units)
-            for u in list(range(n_units)) + list(reversed(range(n_units))):
-                Z.zero_gather_layer(self.lp, u, self.params, self.layer[:self.units[u][0]], stream)
-                Z.zero_release_layer(self.lp, u)
+            self.gathers(stream)
+
+    def gathers(self, stream):
+        """Stage 3: every unit materialised in forward order, then in reverse
+        (each released at once); with a prefetch window the next `prefetch`
+        units are gathered on a side stream meanwhile."""
+        Z = self.Z
+        n_units = len(self.units)
+        fwd, bwd = list(range(n_units)), list(reversed(range(n_units)))
+        if self.prefetch:
+            from zero_partitioned_optimizer_step_b200.prefetch import walk_layers
+            for order in (fwd, bwd):
+                walk_layers(self.lp, self.params, order, lambda u, x: None, depth=self.prefetch,
+                            buffers=self.ring, stream=stream, side_stream=self.side)
+            return
+        for u in fwd + bwd:
+            Z.zero_gather_layer(self.lp, u, self.params, self.layer[:self.units[u][0]], stream)
+            Z.zero_release_layer(self.lp, u)
 
     def _make_chunks(self):
         """Bucket ranges that each hold exactly one bucket with work for this
@@ -411,7 +451,7 @@ def run_ours(args, cfg, rank, world, dist):
     import torch
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    wl = Workload(cfg, dev)
+    wl = Workload(cfg, dev, prefetch=args.prefetch, weight_decay=args.weight_decay)
     stream = torch.cuda.current_stream(dev)
     # warm-up (also builds the per-device launch grid)
     t = 1
@@ -419,7 +459,9 @@ def run_ours(args, cfg, rank, world, dist):
         wl.step(t, stream)
         t += 1
     sg = None
-    if args.graph:
+    if args.graph and args.eager:
+        raise SystemExit("--graph and --eager exclude each other")
+    if args.graph or (not args.eager and wl.layer is None):
         sg = wl.make_graph()
         for _ in range(args.warmup):
             sg.replay(t)
@@ -472,7 +514,117 @@ def run_ours(args, cfg, rank, world, dist):
         return None
     res = _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=n_ev)
     res["config"]["graph"] = sg is not None
+    res["config"]["weight_decay"] = args.weight_decay
+    if wl.layer is not None:
+        Z = wl.Z
+        res["config"].update(prefetch=args.prefetch or 0,
+                             peak_live_units=wl.lp.query(Z.ZERO_Q_PEAK_LIVE_UNITS),
+                             peak_live_bytes=wl.lp.query(Z.ZERO_Q_PEAK_LIVE_BYTES))
     return res
+
+
+def guarded_launches(lp):
+    """Kernels zero_step_guarded launches per step (all-ranks view): per
+    bucket an unaligned head, an 8-aligned body and a tail in each pass (one
+    scalar launch where the bucket's offsets are not multiples of 8), and the
+    one-block finalize between the passes."""
+    import zero_partitioned_optimizer_step_b200 as Z
+    units = lp.units()
+    multi = len(units) > 1
+    n = 0
+    for b in range(lp.n_buckets):
+        u = lp.query(Z.ZERO_Q_BUCKET_UNIT, b)
+        _, _, s, U, O = units[u]
+        j0, j1 = lp.query(Z.ZERO_Q_BUCKET_BEGIN, b) - U, lp.query(Z.ZERO_Q_BUCKET_END, b) - U
+        vec = U % 8 == 0 and O % 8 == 0 and (not multi or (s % 8 == 0 and (lp.S - s) % 8 == 0))
+        lo, hi = (j0 + 7) // 8 * 8, j1 // 8 * 8
+        n += 1 if (not vec or lo >= hi) else (j0 < lo) + 1 + (hi < j1)
+    return 2 * n + 1
+
+
+def run_guarded(args, cfg, rank, world, dist):
+    """--guarded: the two-pass step with global-norm clipping (at
+    --max-grad-norm) and skipping on non-finite gradients, zero_step_guarded,
+    on the workload's buffers (stage 3 adds the layer gathers, as in the
+    plain step).  Its roofline is the whole guarded call: pass 1 reads the Nd
+    bf16 rows and writes the fp32 sum, pass 2 reads the sum and w, m, v and
+    writes w, m, v and the parameters."""
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = Workload(cfg, dev, prefetch=args.prefetch, weight_decay=args.weight_decay)
+    if wl.owner >= 0:
+        raise SystemExit("--guarded: the one-owner view has no global norm; pick an all-ranks workload")
+    Z = wl.Z
+    red = torch.empty(wl.lp.nd * wl.S, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        Z.zero_step_guarded(wl.lp, wl.G, wl.w, wl.m, wl.v, wl.params, wl.adam, t,
+                            max_grad_norm=args.max_grad_norm, skip_nonfinite=True,
+                            reduced_grad=red, grad_norm_sq=wl.norm, overflow=wl.ovf,
+                            workspace=wl.ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if wl.layer is not None:
+            wl.gathers(stream)
+
+    t = 1
+    for _ in range(args.warmup):
+        step(t)
+        t += 1
+    Z.zero_stream_status()
+    events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index).start()
+    time.sleep(0.2)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for k in range(args.steps):
+        step(t + k, events[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    Z.zero_stream_status()
+    skipped = int(wl.ovf.item())
+    elapsed = max_over_ranks(start.elapsed_time(end) / 1e3, dist, dev)
+    g_time = max_over_ranks(sum(a.elapsed_time(b) for a, b in events) / 1e3, dist, dev)
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    g_bytes = Z.zero_bytes_moved(wl.lp, Z.ZERO_BYTES_HBM_GUARDED_STEP)
+    step_bytes = g_bytes + wl.gather_bytes
+    achieved = g_bytes * args.steps / g_time / 1e9
+    return {
+        "metric": METRIC, "value": job_value(world, wl.params_per_step, args.steps, elapsed),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg["workload"] + ", guarded step (clip at %g, skip on overflow)"
+                               % args.max_grad_norm,
+                   "psi": cfg["psi"], "nd": cfg["nd"], "stage": cfg["stage"],
+                   "bucket_elems": cfg["bucket_elems"], "guarded": True,
+                   "max_grad_norm": args.max_grad_norm, "last_step_skipped": bool(skipped),
+                   "hbm_bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (step_bytes / 1e9)},
+        "hbm_gbs": step_bytes / (elapsed / args.steps) / 1e9,
+        "roofline": {"kernel": "guarded step (k_reduce, k_guard_finalize, k_apply: the whole call)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
+                     "traffic": None, "algorithmic_bytes_per_call": g_bytes,
+                     "avg_call_ms": g_time / args.steps * 1e3},
+        "e2e": None,
+        "gpu_launches": (guarded_launches(wl.lp) + (2 * len(wl.units) if wl.layer is not None else 0))
+                        * args.steps,
+        "clocks": clk,
+    }
 
 
 def _e2e(args, wl, stream, dev, world, dist, t_first):
@@ -568,7 +720,8 @@ def run_peer(args, cfg, rank, world, dist):
     units = lp.units()
     unit_len, unit_pad = [u[0] for u in units], [u[1] for u in units]
     S, psi_pad = lp.S, lp.psi_pad
-    adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd)
+    adam = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=1.0 / nd,
+                weight_decay=args.weight_decay)
     w_log = inputs.master_logical(unit_len, unit_pad, cfg["seed_id"], dev)
     ranks = range(nd) if world == 1 else [rank]
     R = {}
@@ -664,6 +817,7 @@ def run_peer(args, cfg, rank, world, dist):
                    "bucket_elems": cfg["bucket_elems"], "peer": True,
                    "hbm_bytes_per_step": hbm_step,
                    "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (hbm_step / 1e9)},
+        "hbm_gbs": hbm_step / (elapsed / args.steps) / 1e9,
         "roofline": roof, "e2e": None,
         "gpu_launches": sum(peer_launches(lp, r) for r in ranks) * args.steps, "clocks": clk,
     }
@@ -691,6 +845,68 @@ def peer_launches(lp, r):
         else:
             n += (p0 < vlo) + 1 + (vhi < p1)
     return n + 1
+
+
+def run_reshard(args, cfg, rank, world, dist):
+    """--reshard ND2: the checkpoint step that moves the workload's owner
+    storage (fp32 w, m, v, and at stage 3 the bf16 parameter shards) from its
+    Nd ranks to ND2 ranks (zero_reshard, one call per array), timed over
+    --steps repetitions.  Algorithmic bytes: every real element read once
+    and every element of the new layout (padding included) written once."""
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = Workload(cfg, dev)
+    if wl.owner >= 0:
+        raise SystemExit("--reshard: the one-owner view holds one rank's shard only")
+    Z = wl.Z
+    to = Z.zero_plan(cfg["psi"], args.reshard, cfg["stage"], cfg["bucket_elems"], unit_elems=cfg["units"])
+    arrays = [wl.w, wl.m, wl.v] + ([wl.params] if cfg["stage"] == 3 else [])
+    outs = [torch.empty(to.nd * to.S, dtype=x.dtype, device=dev) for x in arrays]
+    real = sum(u[0] for u in wl.units)
+    nbytes = sum((real + to.nd * to.S) * x.element_size() for x in arrays)
+    stream = torch.cuda.current_stream(dev)
+
+    def once():
+        for x, y in zip(arrays, outs):
+            Z.zero_reshard(wl.lp, x, to, y, stream=stream)
+
+    for _ in range(args.warmup):
+        once()
+    Z.zero_stream_status()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index).start()
+    time.sleep(0.2)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        once()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    Z.zero_stream_status()
+    elapsed = max_over_ranks(start.elapsed_time(end) / 1e3, dist, dev)
+    if rank != 0:
+        return None
+    peak, peak_kind = measured_peak()
+    achieved = nbytes * args.steps / elapsed / 1e9
+    return {
+        "metric": "Gparams/s resharded (owner storage, Nd to ND2)", "unit": UNIT,
+        "value": job_value(world, cfg["psi"], args.steps, elapsed), "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg["workload"] + ", reshard Nd=%d -> %d" % (cfg["nd"], args.reshard),
+                   "psi": cfg["psi"], "nd": cfg["nd"], "nd_to": args.reshard, "stage": cfg["stage"],
+                   "arrays": len(arrays), "hbm_bytes_per_step": nbytes},
+        "hbm_gbs": achieved,
+        "roofline": {"kernel": "k_reshard (one launch per unit and array)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind + " (copy bandwidth)", "traffic": None},
+        "e2e": None,
+        "gpu_launches": len(arrays) * len(wl.units) * args.steps,
+        "clocks": clk,
+    }
 
 
 def run_sweep(args, rank, world, dist):
@@ -780,7 +996,9 @@ def main():
         if args.sweep:
             run_sweep(args, rank, world, dist)
             return 0
-        res = (run_peer if args.peer else run_ours)(args, cfg, rank, world, dist)
+        run = (run_peer if args.peer else run_guarded if args.guarded else
+               run_reshard if args.reshard else run_ours)
+        res = run(args, cfg, rank, world, dist)
         if res is not None:
             print(json.dumps(res), flush=True)
     finally:

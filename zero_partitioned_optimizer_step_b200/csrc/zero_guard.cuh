@@ -32,8 +32,13 @@ __device__ __forceinline__ uint64_t owner_of(const StepArgs &a, uint64_t j, bool
     return owner_map ? j / a.shard : 0;
 }
 
+// CTAs per SM the two passes are sized for (registers <= 64 per thread).
+constexpr int kGuardMinB = 4;
+// Gradient rows of pass 1 loaded together before their in-order adds.
+constexpr int kGuardRB = 8;
+
 template <int VEC, bool OWNER_MAP>
-__global__ void __launch_bounds__(kThreads) k_reduce(const StepArgs a) {
+__global__ void __launch_bounds__(kThreads, kGuardMinB) k_reduce(const StepArgs a) {
     const uint64_t n = (a.j1 - a.j0) / VEC;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
     double acc = 0.0;
@@ -46,18 +51,18 @@ __global__ void __launch_bounds__(kThreads) k_reduce(const StepArgs a) {
         float s[VEC];
         if constexpr (VEC == 8) {
             const uint16_t *g = a.grads + gi;
-            uint4 x[4];
-            zero_dev::unpack8(__ldcs(reinterpret_cast<const uint4 *>(g)), s);
-            uint32_t r = 1;
-            for (; r + 4 <= a.nd; r += 4) {
+            for (uint32_t r0 = 0; r0 < a.nd; r0 += kGuardRB) {
+                uint4 x[kGuardRB];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    x[k] = __ldcs(reinterpret_cast<const uint4 *>(g + uint64_t(r + k) * a.grad_stride));
+                for (int k = 0; k < kGuardRB; ++k)
+                    if (r0 + k < a.nd) x[k] = __ldcs(reinterpret_cast<const uint4 *>(g + uint64_t(r0 + k) * a.grad_stride));
 #pragma unroll
-                for (int k = 0; k < 4; ++k) zero_dev::add8(s, x[k]);
+                for (int k = 0; k < kGuardRB; ++k) {  // rank order, from rank 0's value
+                    if (r0 + k >= a.nd) break;
+                    if (r0 + k == 0) zero_dev::unpack8(x[0], s);
+                    else zero_dev::add8(s, x[k]);
+                }
             }
-            for (; r < a.nd; ++r)
-                zero_dev::add8(s, __ldcs(reinterpret_cast<const uint4 *>(g + uint64_t(r) * a.grad_stride)));
             __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(s[0], s[1], s[2], s[3]));
             __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(s[4], s[5], s[6], s[7]));
         } else {
@@ -114,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) k_guard_finalize(const double *ws_no
 }
 
 template <int VEC, bool OWNER_MAP>
-__global__ void __launch_bounds__(kThreads) k_apply(const StepArgs a, const GuardWord *gw) {
+__global__ void __launch_bounds__(kThreads, kGuardMinB) k_apply(const StepArgs a, const GuardWord *gw) {
     const GuardWord g = *gw;
     if (g.skip) return;
     const AdamConsts C = zero_dev::consts_of(a);

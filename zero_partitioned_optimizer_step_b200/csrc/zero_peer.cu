@@ -45,9 +45,13 @@
 #include <utility>
 
 #include "zero_device.cuh"
+#include "zero_host.cuh"
 #include "zero_internal.h"
 
 using zero_detail::set_error;
+using zero_host::aligned16;
+using zero_host::check_launch;
+using zero_host::mult8;
 
 namespace {
 
@@ -231,15 +235,6 @@ __global__ void __launch_bounds__(kThreads) k_gather_peer(const PeerTable T, uin
 }
 
 // ----------------------------------------------------------------- host side
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool mult8(int64_t x) { return (uint64_t(x) & 7u) == 0; }
-
-zero_status_t check_launch(const char *what) {
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
-    return ZERO_OK;
-}
 
 // Launch shapes on the current device, computed once per device: the
 // persistent grid of the peer step kernels (SM count x resident CTAs, capped

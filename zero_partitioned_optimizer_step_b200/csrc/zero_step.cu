@@ -45,9 +45,13 @@
 #include "zero_device.cuh"
 #include "zero_guard.cuh"
 #include "zero_tma.cuh"
+#include "zero_host.cuh"
 #include "zero_internal.h"
 
 using zero_detail::set_error;
+using zero_host::aligned16;
+using zero_host::check_launch;
+using zero_host::mult8;
 
 namespace {
 
@@ -224,8 +228,6 @@ __global__ void __launch_bounds__(kThreads) k_gather(const uint16_t *src, uint64
 
 // ----------------------------------------------------------------- host side
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 // The bulk-copy kernel instantiations: owner map x consumer groups x vector width.
 using TmaKernel = void (*)(const StepArgs, const zero_tma::Ring);
 
@@ -245,6 +247,7 @@ TmaKernel tma_kernel(uint32_t groups, uint32_t vw) {
 // shared memory the bulk-copy kernel may use.
 struct DeviceShapes {
     uint32_t grid_ldg = 0;
+    uint32_t grid_guard = 0;  // the guarded step's two passes (fewer registers)
     uint32_t sms = 0;
     uint32_t tma_smem = 0;
 };
@@ -261,16 +264,21 @@ zero_status_t device_shapes(DeviceShapes *out) {
         *out = it->second;
         return ZERO_OK;
     }
-    int sms = 0, occ = 0, optin = 0;
+    int sms = 0, occ = 0, optin = 0, occ_r = 0, occ_a = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_vec8<false, kRB, kMinB>, kThreads, 0);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_r, zero_guarded::k_reduce<8, true>, kThreads, 0);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, zero_guarded::k_apply<8, true>, kThreads, 0);
     cudaFuncAttributes fa{};
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
     DeviceShapes d;
     d.sms = uint32_t(std::max(1, sms));
     d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
+    d.grid_guard = std::min(uint32_t(std::max(1, sms) * std::max(1, std::min(occ_r, occ_a))), zero_detail::kMaxSlots);
     const int64_t budget = int64_t(optin) - int64_t(fa.sharedSizeBytes) - 256;
     d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
     if (d.tma_smem > 0) {
@@ -392,14 +400,6 @@ AdamConsts make_consts(const zero_adam_t &a, uint64_t t) {
     c.decay = float(1.0 - a.lr * a.weight_decay);
     return c;
 }
-
-zero_status_t check_launch(const char *what) {
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
-    return ZERO_OK;
-}
-
-bool mult8(int64_t x) { return (uint64_t(x) & 7u) == 0; }
 
 // Launch with or without programmatic dependent launch on the stream.
 template <typename... Params, typename... Args>
@@ -742,7 +742,7 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     cudaError_t e = cudaMemsetAsync(b->workspace, 0, zero_detail::kWorkspaceBytes, stream);
     if (e != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("zero_step_guarded workspace reset: ") + cudaGetErrorString(e));
-    const uint32_t grid = shapes.grid_ldg;
+    const uint32_t grid = shapes.grid_guard;
     // pass 1: reductions, sums of squares, non-finite counts
     for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
         StepArgs x;
@@ -781,68 +781,6 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             else zero_guarded::k_apply<1, false><<<grid, kThreads, 0, stream>>>(y, gw);
             return check_launch("zero_step_guarded apply launch");
         });
-        if (st != ZERO_OK) return st;
-    }
-    return ZERO_OK;
-}
-
-// ------------------------------------------------------------- resharding
-namespace {
-
-// K4: one unit's elements from owner storage under plan A to owner storage
-// under plan B (same unit lengths, other Nd or padding).  Thread per
-// destination element q of the unit's slices: owner o' = q / s'_u,
-// logical j = o' * s'_u + (q mod s'_u); j >= len_u is padding (zero).
-template <typename T>
-__global__ void __launch_bounds__(kThreads) k_reshard(const T *src, uint64_t S_a, uint64_t off_a, uint64_t s_a,
-                                                     T *dst, uint64_t S_b, uint64_t off_b, uint64_t s_b,
-                                                     uint32_t nd_b, uint64_t len) {
-    const uint64_t n = uint64_t(nd_b) * s_b;
-    const uint64_t stride = uint64_t(gridDim.x) * kThreads;
-    for (uint64_t q = uint64_t(blockIdx.x) * kThreads + threadIdx.x; q < n; q += stride) {
-        const uint64_t ob = q / s_b, i = q - ob * s_b;
-        const uint64_t j = q;  // logical index inside the unit (ob * s_b + i)
-        T val = T(0);
-        if (j < len) {
-            const uint64_t oa = j / s_a;
-            val = src[oa * S_a + off_a + (j - oa * s_a)];
-        }
-        dst[ob * S_b + off_b + i] = val;
-    }
-}
-
-}  // namespace
-
-ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, const zero_plan_t *to, void *dst,
-                                    uint32_t elem_bytes, void *stream_) {
-    zero_detail::clear_error();
-    if (!from || !to || !src || !dst) return set_error(ZERO_EINVAL, "zero_reshard: NULL argument");
-    if (elem_bytes != 2 && elem_bytes != 4)
-        return set_error(ZERO_EINVAL, "zero_reshard: elem_bytes must be 2 (bf16) or 4 (fp32)");
-    if (from->unit_len != to->unit_len)
-        return set_error(ZERO_EINVAL, "zero_reshard: the two plans must have the same unit lengths");
-    if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) % elem_bytes)
-        return set_error(ZERO_EINVAL, "zero_reshard: buffers must be aligned to the element size");
-    cudaError_t pre = cudaPeekAtLastError();
-    if (pre != cudaSuccess)
-        return set_error(ZERO_ECUDA, std::string("pending CUDA error before zero_reshard: ") +
-                                         cudaGetErrorString(pre));
-    DeviceShapes shapes;
-    zero_status_t st = device_shapes(&shapes);
-    if (st != ZERO_OK) return st;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
-    for (size_t u = 0; u < to->unit_len.size(); ++u) {
-        const uint64_t n = uint64_t(to->nd) * to->unit_shard[u];
-        const uint32_t grid = uint32_t(std::min<uint64_t>((n + kThreads - 1) / kThreads, uint64_t(shapes.sms) * 8));
-        if (elem_bytes == 4)
-            k_reshard<uint32_t><<<grid, kThreads, 0, stream>>>(
-                static_cast<const uint32_t *>(src), from->S, from->unit_offset[u], from->unit_shard[u],
-                static_cast<uint32_t *>(dst), to->S, to->unit_offset[u], to->unit_shard[u], to->nd, to->unit_len[u]);
-        else
-            k_reshard<uint16_t><<<grid, kThreads, 0, stream>>>(
-                static_cast<const uint16_t *>(src), from->S, from->unit_offset[u], from->unit_shard[u],
-                static_cast<uint16_t *>(dst), to->S, to->unit_offset[u], to->unit_shard[u], to->nd, to->unit_len[u]);
-        st = check_launch("zero_reshard launch");
         if (st != ZERO_OK) return st;
     }
     return ZERO_OK;
