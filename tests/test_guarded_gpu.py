@@ -84,3 +84,21 @@ def test_guarded_requires_its_buffers():
         Z.zero_step_guarded(c.lp, c.grads(1), c.w, c.m, c.v, c.params, c.adam, 1,
                             max_grad_norm=-1.0, reduced_grad=c.red, grad_norm_sq=c.norm,
                             overflow=c.ovf, workspace=c.ws)
+
+
+@pytest.mark.parametrize("offset", [0, 4])
+def test_guarded_state_at_16_byte_offsets(offset):
+    """The fp32 arrays 32-byte aligned (32-byte accesses) or only 16-byte
+    aligned (16-byte accesses): the same bits."""
+    psi, nd = 500_000, 8
+    c = Case(psi, nd, 2, 1 << 15, config_id=15, adam=ADAMW)
+    for name in ("w", "m", "v", "red"):
+        x = getattr(c, name)
+        big = torch.empty(x.numel() + 8, dtype=x.dtype, device="cuda")
+        y = big[offset:offset + x.numel()]
+        y.copy_(x)
+        setattr(c, name, y)
+    assert (c.w.data_ptr() % 32 == 0) == (offset == 0)
+    for t in (1, 2):
+        diff, coef, skipped = c.guarded_step_and_compare(t, 0.05, True)
+        assert 0 < coef < 1 and not skipped

@@ -32,12 +32,27 @@ __device__ __forceinline__ uint64_t owner_of(const StepArgs &a, uint64_t j, bool
     return owner_map ? j / a.shard : 0;
 }
 
+// 8 consecutive fp32 with one 32-byte access (sm_100 and later; the address
+// must be 32-byte aligned), streaming cache hint.
+__device__ __forceinline__ void ld8_cs(const float *p, float f[8]) {
+    asm volatile("ld.global.cs.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=f"(f[0]), "=f"(f[1]), "=f"(f[2]), "=f"(f[3]), "=f"(f[4]), "=f"(f[5]), "=f"(f[6]), "=f"(f[7])
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void st8_cs(float *p, const float f[8]) {
+    asm volatile("st.global.cs.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(f[0]), "f"(f[1]),
+                 "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7])
+                 : "memory");
+}
+
 // CTAs per SM the two passes are sized for (registers <= 64 per thread).
 constexpr int kGuardMinB = 4;
 // Gradient rows of pass 1 loaded together before their in-order adds.
 constexpr int kGuardRB = 8;
 
-template <int VEC, bool OWNER_MAP>
+// W32: the fp32 arrays are 32-byte aligned (one 32-byte access per 8 elements).
+template <int VEC, bool OWNER_MAP, bool W32 = false>
 __global__ void __launch_bounds__(kThreads, kGuardMinB) k_reduce(const StepArgs a) {
     const uint64_t n = (a.j1 - a.j0) / VEC;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
@@ -63,8 +78,12 @@ __global__ void __launch_bounds__(kThreads, kGuardMinB) k_reduce(const StepArgs 
                     else zero_dev::add8(s, x[k]);
                 }
             }
-            __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(s[0], s[1], s[2], s[3]));
-            __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(s[4], s[5], s[6], s[7]));
+            if constexpr (W32) {
+                st8_cs(a.red + si, s);
+            } else {
+                __stcs(reinterpret_cast<float4 *>(a.red + si), make_float4(s[0], s[1], s[2], s[3]));
+                __stcs(reinterpret_cast<float4 *>(a.red + si + 4), make_float4(s[4], s[5], s[6], s[7]));
+            }
         } else {
             s[0] = __uint_as_float(uint32_t(a.grads[gi]) << 16);
             for (uint32_t r = 1; r < a.nd; ++r)
@@ -118,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) k_guard_finalize(const double *ws_no
     }
 }
 
-template <int VEC, bool OWNER_MAP>
+template <int VEC, bool OWNER_MAP, bool W32 = false>
 __global__ void __launch_bounds__(kThreads, kGuardMinB) k_apply(const StepArgs a, const GuardWord *gw) {
     const GuardWord g = *gw;
     if (g.skip) return;
@@ -130,7 +149,25 @@ __global__ void __launch_bounds__(kThreads, kGuardMinB) k_apply(const StepArgs a
         const uint64_t o = owner_of(a, j, OWNER_MAP);
         const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
         const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
-        if constexpr (VEC == 8) {
+        if constexpr (VEC == 8 && W32) {
+            float s[8], w[8], m[8], v[8];
+            ld8_cs(a.red + si, s);
+            ld8_cs(a.w + si, w);
+            ld8_cs(a.m + si, m);
+            ld8_cs(a.v + si, v);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) zero_dev::adam1c(s[e], g.coef, C, w[e], m[e], v[e]);
+            st8_cs(a.w + si, w);
+            st8_cs(a.m + si, m);
+            st8_cs(a.v + si, v);
+            uint4 pk;
+            pk.x = zero_dev::pack_bf16x2(w[0], w[1]);
+            pk.y = zero_dev::pack_bf16x2(w[2], w[3]);
+            pk.z = zero_dev::pack_bf16x2(w[4], w[5]);
+            pk.w = zero_dev::pack_bf16x2(w[6], w[7]);
+            for (uint32_t r = 0; r < a.n_prow; ++r)
+                __stcs(reinterpret_cast<uint4 *>(a.params + pi + uint64_t(r) * a.param_stride), pk);
+        } else if constexpr (VEC == 8) {
             float s[8], w[8], m[8], v[8];
             const float4 *rp = reinterpret_cast<const float4 *>(a.red + si);
             const float4 *wp = reinterpret_cast<const float4 *>(a.w + si);

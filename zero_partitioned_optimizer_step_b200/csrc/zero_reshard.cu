@@ -24,10 +24,11 @@ using zero_dev::kThreads;
 // (jump = S - s_u), and under plan A at off_a + q + oa * jump_a, oa = q / s_a;
 // q >= len is padding, written as zero.  A warp copies chunks of 32 * V * R
 // consecutive q: lane l takes the groups of V elements at l*V, l*V + 32V, ...,
-// so the warp's accesses are contiguous, and the two owners, found by one
-// division per chunk, only advance within it.  V = 16 bytes of elements when
-// every offset, shard and jump is a multiple of V, else 1 (a group of V never
-// straddles a shard boundary then).
+// so the warp's accesses are contiguous.  The two owners, found by one
+// division per chunk, only advance within it.  A lane issues all R loads of
+// its chunk before any of its stores, so R loads are in flight at once.
+// V = 16 bytes of elements when every offset, shard and jump is a multiple of
+// V, else 1 (a group of V then never straddles a shard boundary).
 struct ReshardArgs {
     uint64_t off_a, jump_a, s_a;
     uint64_t off_b, jump_b, s_b;
@@ -50,13 +51,17 @@ __global__ void __launch_bounds__(kThreads) k_reshard(const T *__restrict__ src,
     const uint64_t warp = (uint64_t(blockIdx.x) * kThreads + threadIdx.x) >> 5;
     const uint64_t nwarps = (uint64_t(gridDim.x) * kThreads) >> 5;
     for (uint64_t c0 = warp * kChunk; c0 < a.n; c0 += nwarps * kChunk) {
-        uint64_t q = c0 + uint64_t(lane) * V;
-        if (q >= a.n) continue;
-        uint64_t oa = q / a.s_a, ob = q / a.s_b;
+        const uint64_t q0 = c0 + uint64_t(lane) * V;
+        if (q0 >= a.n) continue;
+        uint64_t oa = q0 / a.s_a, ob = q0 / a.s_b;
         uint64_t na = (oa + 1) * a.s_a, nb = (ob + 1) * a.s_b;  // next shard boundaries
-#pragma unroll 4
-        for (int k = 0; k < R; ++k, q += 32ull * V) {
-            if (q >= a.n) break;
+        VT val[R];
+        uint64_t sp[R], dp[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const uint64_t q = q0 + uint64_t(k) * 32 * V;
+            sp[k] = dp[k] = ~uint64_t(0);
+            if (q >= a.n) continue;
             while (q >= na) {
                 ++oa;
                 na += a.s_a;
@@ -65,13 +70,20 @@ __global__ void __launch_bounds__(kThreads) k_reshard(const T *__restrict__ src,
                 ++ob;
                 nb += a.s_b;
             }
-            T *d = dst + a.off_b + q + ob * a.jump_b;
-            const T *s = src + a.off_a + q + oa * a.jump_a;
-            if (q + V <= a.len) {
-                __stcs(reinterpret_cast<VT *>(d), __ldcs(reinterpret_cast<const VT *>(s)));
-            } else {
+            sp[k] = a.off_a + q + oa * a.jump_a;
+            dp[k] = a.off_b + q + ob * a.jump_b;
+            if (q + V <= a.len) val[k] = __ldcs(reinterpret_cast<const VT *>(src + sp[k]));
+        }
 #pragma unroll
-                for (int e = 0; e < V; ++e) d[e] = q + e < a.len ? s[e] : T(0);
+        for (int k = 0; k < R; ++k) {
+            const uint64_t q = q0 + uint64_t(k) * 32 * V;
+            if (q >= a.n) continue;
+            T *d = dst + dp[k];
+            if (q + V <= a.len) {
+                __stcs(reinterpret_cast<VT *>(d), val[k]);
+            } else {  // the group holding the end of the unit, or padding
+#pragma unroll
+                for (int e = 0; e < V; ++e) d[e] = q + e < a.len ? src[sp[k] + e] : T(0);
             }
         }
     }
@@ -108,7 +120,7 @@ ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, co
         r.len = to->unit_len[u];
         const uint64_t V = 16 / elem_bytes;
         const bool vec = vec_bytes && ((r.off_a | r.s_a | r.jump_a | r.off_b | r.s_b | r.jump_b) % V) == 0;
-        constexpr int R = 16;
+        constexpr int R = 8;
         const uint64_t per_thread = (vec ? V : 1) * R;
         const uint64_t blocks = (r.n + per_thread * kThreads - 1) / (per_thread * kThreads);
         const uint32_t grid = uint32_t(std::max<uint64_t>(1, std::min<uint64_t>(blocks, uint64_t(sms) * 8)));

@@ -270,9 +270,9 @@ zero_status_t device_shapes(DeviceShapes *out) {
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_vec8<false, kRB, kMinB>, kThreads, 0);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_r, zero_guarded::k_reduce<8, true>, kThreads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_r, zero_guarded::k_reduce<8, true, true>, kThreads, 0);
     if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, zero_guarded::k_apply<8, true>, kThreads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, zero_guarded::k_apply<8, true, true>, kThreads, 0);
     cudaFuncAttributes fa{};
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
     DeviceShapes d;
@@ -743,6 +743,10 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     if (e != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("zero_step_guarded workspace reset: ") + cudaGetErrorString(e));
     const uint32_t grid = shapes.grid_guard;
+    // fp32 arrays 32-byte aligned: 32-byte accesses on the vector path
+    const bool w32 = ((reinterpret_cast<uintptr_t>(b->master) | reinterpret_cast<uintptr_t>(b->exp_avg) |
+                       reinterpret_cast<uintptr_t>(b->exp_avg_sq) | reinterpret_cast<uintptr_t>(b->reduced_grad)) &
+                      31u) == 0;
     // pass 1: reductions, sums of squares, non-finite counts
     for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
         StepArgs x;
@@ -752,7 +756,9 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             StepArgs y = x;
             y.j0 = j0;
             y.j1 = j1;
-            if (vec && om) zero_guarded::k_reduce<8, true><<<grid, kThreads, 0, stream>>>(y);
+            if (vec && om && w32) zero_guarded::k_reduce<8, true, true><<<grid, kThreads, 0, stream>>>(y);
+            else if (vec && w32) zero_guarded::k_reduce<8, false, true><<<grid, kThreads, 0, stream>>>(y);
+            else if (vec && om) zero_guarded::k_reduce<8, true><<<grid, kThreads, 0, stream>>>(y);
             else if (vec) zero_guarded::k_reduce<8, false><<<grid, kThreads, 0, stream>>>(y);
             else if (om) zero_guarded::k_reduce<1, true><<<grid, kThreads, 0, stream>>>(y);
             else zero_guarded::k_reduce<1, false><<<grid, kThreads, 0, stream>>>(y);
@@ -775,7 +781,9 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             StepArgs y = x;
             y.j0 = j0;
             y.j1 = j1;
-            if (vec && om) zero_guarded::k_apply<8, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            if (vec && om && w32) zero_guarded::k_apply<8, true, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            else if (vec && w32) zero_guarded::k_apply<8, false, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            else if (vec && om) zero_guarded::k_apply<8, true><<<grid, kThreads, 0, stream>>>(y, gw);
             else if (vec) zero_guarded::k_apply<8, false><<<grid, kThreads, 0, stream>>>(y, gw);
             else if (om) zero_guarded::k_apply<1, true><<<grid, kThreads, 0, stream>>>(y, gw);
             else zero_guarded::k_apply<1, false><<<grid, kThreads, 0, stream>>>(y, gw);
