@@ -59,8 +59,8 @@
  * unaligned heads and tails in a scalar kernel.  All give identical results.
  * The environment variable ZERO_STEP_KERNEL=ldg|tma overrides the choice.
  * The bulk-copy kernel's shared-memory ring is sized per Nd; for a bucket of
- * fewer than 32 tiles per SM it is cut to half of an SM's shared memory, so
- * that the next bucket's CTAs share the SM.  Bucket kernels after the first
+ * fewer than 32 x 2048 elements per SM it is cut to half of an SM's shared
+ * memory, so that the next bucket's CTAs share the SM.  Bucket kernels after the first
  * of a call use programmatic dependent launch.  Tuning switches (results do
  * not change): ZERO_TMA_TILE, ZERO_TMA_STAGES, ZERO_TMA_GROUPS, ZERO_TMA_VW,
  * ZERO_TMA_ADAPT=0, ZERO_TMA_ADAPT_TILES, ZERO_LDG_RB=4|8, ZERO_PDL=0.

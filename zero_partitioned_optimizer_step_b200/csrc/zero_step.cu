@@ -301,7 +301,7 @@ uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
 // tile pays a fixed synchronisation latency, so tiles are large; two consumer
 // groups help where a tile is cheap to compute.  Shapes measured best on B200
 // at 64 MB buckets (5e8 params), as (groups, tile, stages, elements/thread):
-//   Nd <= 4: (2, 2048, 4, 8)     Nd <= 8: (1, 2048, 3, 8)
+//   Nd <= 2: (2, 2048, 4, 8)     Nd <= 4: (1, 4096, 2, 8)     Nd <= 8: (1, 2048, 3, 8)
 //   Nd <= 16: (1, 1024, 4, 4)    Nd <= 32: (1, 1024, 2, 8)
 //   Nd <= 64: (1, 512, 3, 4)
 // Read-heavy steps (parameters written once: stage 3 or one owner) do better
@@ -340,8 +340,10 @@ bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, zero_tma::Ring *
         stages = force_s >= 2 ? uint32_t(std::min<long>(force_s, zero_tma::kMaxStages)) : zero_tma::kMaxStages;
         const uint64_t busy = tile * groups / zero_tma::kConsumers;  // keep a group's threads busy
         vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
-    } else if (nd <= 4) {
+    } else if (nd <= 2) {
         groups = 2, tile = 2048, stages = 4, vw = 8;
+    } else if (nd <= 4) {
+        groups = 1, tile = 4096, stages = 2, vw = 8;
     } else if (nd <= 8) {
         groups = 1, tile = 2048, stages = 3, vw = 8;
     } else if (nd <= 16 && read_heavy) {
@@ -376,14 +378,15 @@ bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, zero_tma::Ring *
 
 // A small bucket is over soon after a CTA's ring has filled, and the next
 // bucket's CTAs (launched early through programmatic dependent launch) cannot
-// start on an SM while this ring takes most of its shared memory.  Below 32
-// tiles per SM the ring is cut to half of the SM's shared memory (tile
+// start on an SM while this ring takes most of its shared memory.  Below
+// 32 x 2048 elements per SM the ring is cut to half of the SM's shared memory (tile
 // halved while needed, at least 512, and as many stages as then fit), so two
 // CTAs share an SM and the next bucket's loads overlap this one's tail.
 // Measured on B200 (5e8 params): +50 % at 1-2 MB buckets for Nd <= 8 and
 // +10-20 % up to 16 MB; from 32 MB up the full ring is faster.
 // ZERO_TMA_ADAPT=0, or a forced ZERO_TMA_TILE, keeps the chosen ring;
-// ZERO_TMA_ADAPT_TILES=<n> moves the threshold (tuning).
+// ZERO_TMA_ADAPT_TILES=<n> moves the threshold to n x 2048 elements per SM
+// (tuning).
 zero_tma::Ring ring_for_launch(const zero_tma::Ring &r, uint64_t n, uint32_t nd, uint32_t sms,
                                uint32_t budget) {
     static const bool off = [] {
@@ -395,7 +398,7 @@ zero_tma::Ring ring_for_launch(const zero_tma::Ring &r, uint64_t n, uint32_t nd,
         const long v = e ? std::strtol(e, nullptr, 10) : 0;
         return uint64_t(v > 0 ? v : 32);
     }();
-    if (off || n >= uint64_t(r.tile) * per_sm * sms) return r;
+    if (off || n >= 2048ull * per_sm * sms) return r;
     const uint64_t half = budget / 2 - 1024;  // room for a second CTA's ring and static shared memory
     for (uint64_t tile = r.tile; tile >= 512; tile /= 2) {
         zero_tma::Ring q = ring_for(nd, tile, 0, r.groups);
