@@ -46,7 +46,7 @@ UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
 K1_PROFILE = os.path.join(ROOT, "profiles", "k_step_tma_gpt2_small_nd8.md")
 K1_SOURCES = [os.path.join(ROOT, "zero_partitioned_optimizer_step_b200", "csrc", f)
-              for f in ("zero_step.cu", "zero_tma.cuh", "zero_device.cuh")]
+              for f in ("zero_step.cu", "zero_tma.cuh", "zero_ring.cuh", "zero_device.cuh")]
 
 
 def kernel_source_hash():

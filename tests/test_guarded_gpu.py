@@ -32,10 +32,13 @@ def test_adamw_fused_bit_exact(kernel, psi, nd, stage, units, monkeypatch):
         assert all(v == 0 for v in diff.values()), diff
 
 
+@pytest.mark.parametrize("kernel", ["tma", "ldg"])
 @pytest.mark.parametrize("psi,nd,stage,units,align", [
     (500_000, 8, 2, None, 64), (300_001, 16, 3, [100_000, 3, 199_998], 64), (77_777, 5, 1, None, 1)])
-def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align):
-    """A guard that never triggers gives the fused step's bits."""
+def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align, kernel, monkeypatch):
+    """A guard that never triggers gives the fused step's bits (second pass
+    in the bulk-copy kernel, or in the 16-byte-load kernel)."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
     a = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
     b = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
     for t in (1, 2):
@@ -48,9 +51,11 @@ def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align):
         assert torch.equal(a.params.view(torch.int16), b.params.view(torch.int16))
 
 
+@pytest.mark.parametrize("kernel", ["tma", "ldg"])
 @pytest.mark.parametrize("psi,nd,stage,units", [(500_000, 8, 2, None),
                                                 (300_001, 16, 3, [100_000, 3, 199_998])])
-def test_guarded_clipping(psi, nd, stage, units):
+def test_guarded_clipping(psi, nd, stage, units, kernel, monkeypatch):
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
     c = Case(psi, nd, stage, 1 << 15, units=units, sigma=1e-2, config_id=14, adam=ADAMW)
     for t in (1, 2, 3):
         diff, coef, skipped = c.guarded_step_and_compare(t, 0.05, True)

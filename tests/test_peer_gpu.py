@@ -94,8 +94,13 @@ PEER_CASES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", ["tma", "ldg"])
 @pytest.mark.parametrize("psi,nd,stage,bucket,align,units", PEER_CASES)
-def test_ranks_as_allocations_equal_the_one_gpu_step(psi, nd, stage, bucket, align, units):
+def test_ranks_as_allocations_equal_the_one_gpu_step(psi, nd, stage, bucket, align, units, kernel,
+                                                     monkeypatch):
+    """Aligned bodies in the bulk-copy kernel (rows through the peer table)
+    or in K5; both against the one-GPU step."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
     c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=31)
     R = Ranks(c)
     for t in (1, 2, 3):
@@ -237,9 +242,11 @@ def test_two_processes_share_buffers_through_ipc(case):
     assert all(p.exitcode == 0 for p in procs)
 
 
-def test_peer_step_writes_stay_inside_their_buffers():
+@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+def test_peer_step_writes_stay_inside_their_buffers(kernel, monkeypatch):
     """Every rank's buffers inside guard zones of a fixed byte pattern."""
     from test_canary_fuzz_gpu import Guarded
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
     c = Case(100_003, 7, 3, 999, align=1, units=[10_001, 90_002], config_id=34)
     R = Ranks(c)
     guarded = []

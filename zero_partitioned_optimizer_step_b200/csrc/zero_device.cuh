@@ -40,6 +40,21 @@ struct StepArgs {
     int ws_mode;  // 0: no norm; 1: add this launch's per-CTA partials to the slots
 };
 
+// The guarded step's decision, written by its finalize kernel: the clip
+// coefficient (<= 1) and whether to leave the state as it is.
+struct GuardWord {
+    float coef;
+    int32_t skip;
+};
+
+// Device pointers of the Nd ranks when the ranks are devices, passed by
+// value (2 KB of kernel parameters at ZERO_MAX_PEERS = 128).
+constexpr int kMaxPeers = 128;
+struct PeerTable {
+    const uint16_t *g[kMaxPeers];  // rank q's gradient, logical order
+    uint16_t *p[kMaxPeers];        // parameter rows: replicas, or the owner's shard
+};
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

@@ -23,10 +23,7 @@ using zero_dev::AdamConsts;
 using zero_dev::StepArgs;
 using zero_dev::kThreads;
 
-struct GuardWord {
-    float coef;    // clip coefficient, <= 1
-    int32_t skip;  // 1: leave the state as it is
-};
+using zero_dev::GuardWord;
 
 __device__ __forceinline__ uint64_t owner_of(const StepArgs &a, uint64_t j, bool owner_map) {
     return owner_map ? j / a.shard : 0;

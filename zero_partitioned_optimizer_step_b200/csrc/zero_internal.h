@@ -50,6 +50,10 @@ BucketRange bucket_range(const zero_plan_t &p, uint64_t b);
 zero_status_t live_check(const zero_plan_t &p, uint32_t unit, const char *who);
 void live_mark(zero_plan_t &p, uint32_t unit);
 
+// Device address of the current device's error word of the bulk-copy step
+// kernel's bounded waits (what zero_stream_status() reports).
+zero_status_t wait_error_word(int **out);
+
 // Workspace layout for the gradient-norm / overflow reduction: one fp64
 // partial and one u32 count per CTA slot, kMaxSlots slots, then 256 bytes
 // for the guarded step's decision (clip coefficient and skip flag).

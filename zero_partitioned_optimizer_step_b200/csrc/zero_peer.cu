@@ -47,6 +47,8 @@
 #include "zero_device.cuh"
 #include "zero_host.cuh"
 #include "zero_internal.h"
+#include "zero_ring.cuh"
+#include "zero_tma.cuh"
 
 using zero_detail::set_error;
 using zero_host::aligned16;
@@ -60,12 +62,7 @@ using namespace zero_dev;
 constexpr int kPeerMinB = 2;  // CTAs per SM the vector kernel is sized for
 constexpr int kPeerRB = 8;    // gradient rows in flight per thread
 
-// Device pointers of the Nd ranks, passed by value (2 KB of kernel
-// parameters at ZERO_MAX_PEERS).
-struct PeerTable {
-    const uint16_t *g[ZERO_MAX_PEERS];  // rank q's gradient, logical order
-    uint16_t *p[ZERO_MAX_PEERS];        // parameter rows: replicas, or r's shard
-};
+static_assert(kMaxPeers == ZERO_MAX_PEERS, "one peer table size");
 
 // One launch: the logical range [p0, p1) of one unit that rank r owns.
 // State index = p + s_shift; parameter index = p + q_shift (0 for replicas,
@@ -97,8 +94,8 @@ __device__ __forceinline__ void cta_release_system() {
 // adds.  Preconditions (host): p0, p1, s_shift, q_shift multiples of 8 and
 // every pointer 16-byte aligned.
 __global__ void __launch_bounds__(kThreads, kPeerMinB) k_step_peer(const PeerArgs a, const PeerTable T) {
-    __shared__ const uint16_t *sg[ZERO_MAX_PEERS];
-    __shared__ uint16_t *sp[ZERO_MAX_PEERS];
+    __shared__ const uint16_t *sg[kMaxPeers];
+    __shared__ uint16_t *sp[kMaxPeers];
     for (uint32_t i = threadIdx.x; i < a.nd; i += kThreads) sg[i] = T.g[i];
     for (uint32_t i = threadIdx.x; i < a.n_prow; i += kThreads) sp[i] = T.p[i];
     __syncthreads();
@@ -170,8 +167,8 @@ __global__ void __launch_bounds__(kThreads, kPeerMinB) k_step_peer(const PeerArg
 
 // K5, scalar path: any alignment (unit heads and tails, A not a multiple of 8).
 __global__ void __launch_bounds__(kThreads) k_step_peer_scalar(const PeerArgs a, const PeerTable T) {
-    __shared__ const uint16_t *sg[ZERO_MAX_PEERS];
-    __shared__ uint16_t *sp[ZERO_MAX_PEERS];
+    __shared__ const uint16_t *sg[kMaxPeers];
+    __shared__ uint16_t *sp[kMaxPeers];
     for (uint32_t i = threadIdx.x; i < a.nd; i += kThreads) sg[i] = T.g[i];
     for (uint32_t i = threadIdx.x; i < a.n_prow; i += kThreads) sp[i] = T.p[i];
     __syncthreads();
@@ -241,7 +238,20 @@ __global__ void __launch_bounds__(kThreads) k_gather_peer(const PeerTable T, uin
 // at the norm workspace's slot count) and the SM count.
 struct PeerShapes {
     uint32_t grid = 0, sms = 0;
+    uint32_t tma_smem = 0;  // dynamic shared memory the bulk-copy kernel may use
 };
+
+// The bulk-copy kernel with the rows reached through the peer table.
+using PeerTmaKernel = void (*)(const zero_dev::StepArgs, const zero_tma::Ring, const zero_dev::PeerTable);
+
+PeerTmaKernel peer_tma_kernel(uint32_t groups, uint32_t vw) {
+    using namespace zero_tma;
+    if (groups == 2)
+        return vw == 2 ? k_step_tma<false, 2, 2, kPeerRows>
+                       : (vw == 4 ? k_step_tma<false, 2, 4, kPeerRows> : k_step_tma<false, 2, 8, kPeerRows>);
+    return vw == 2 ? k_step_tma<false, 1, 2, kPeerRows>
+                   : (vw == 4 ? k_step_tma<false, 1, 4, kPeerRows> : k_step_tma<false, 1, 8, kPeerRows>);
+}
 
 zero_status_t peer_shapes(PeerShapes *out) {
     static std::mutex mu;
@@ -255,11 +265,22 @@ zero_status_t peer_shapes(PeerShapes *out) {
         *out = it->second;
         return ZERO_OK;
     }
-    int sms = 0, occ = 0;
+    int sms = 0, occ = 0, optin = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_step_peer, kThreads, 0);
-    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("device query: ") + cudaGetErrorString(e));
+    cudaFuncAttributes fa{};
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, peer_tma_kernel(2, 2));
     PeerShapes s;
+    const int64_t budget = int64_t(optin) - int64_t(fa.sharedSizeBytes) - 256;
+    s.tma_smem = budget > 0 ? uint32_t(budget) : 0;
+    if (s.tma_smem > 0)
+        for (uint32_t g : {1u, 2u})
+            for (uint32_t vw : {2u, 4u, 8u})
+                if (e == cudaSuccess)
+                    e = cudaFuncSetAttribute(reinterpret_cast<const void *>(peer_tma_kernel(g, vw)),
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(s.tma_smem));
+    if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("device query: ") + cudaGetErrorString(e));
     s.sms = uint32_t(std::max(1, sms));
     s.grid = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
     cache[dev] = s;
@@ -360,13 +381,51 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
             return set_error(ZERO_ECUDA, std::string("zero_step_peers workspace reset: ") + cudaGetErrorString(e));
     }
 
+    // Aligned bodies run in K5 by default; with ZERO_STEP_KERNEL=tma in the
+    // bulk-copy kernel (rows pulled by 1-D bulk copies through the peer table,
+    // no multicast).  With the ranks as allocations on one GPU K5 is faster
+    // (0.85 against 0.82 of copy bandwidth at Nd = 8, 0.74 against 0.61 for
+    // the stage-3 1.3B workload at Nd = 16: a rank's launches are short); the
+    // NVLink rate of either is not measured.  Unaligned edges: K5's scalar twin.
+    zero_tma::Ring ring{};
+    int *err = nullptr;
+    st = zero_detail::wait_error_word(&err);
+    if (st != ZERO_OK) return st;
+    const bool tma = zero_ring::kernel_choice() == 2 &&
+                     zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring);
     auto launch = [&](uint64_t p0, uint64_t p1, bool vec) -> zero_status_t {
         if (p0 >= p1) return ZERO_OK;
         PeerArgs x = a;
         x.p0 = p0;
         x.p1 = p1;
-        if (vec) k_step_peer<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
-        else k_step_peer_scalar<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
+        if (vec && tma) {
+            StepArgs sa{};
+            sa.w = x.w;
+            sa.m = x.m;
+            sa.v = x.v;
+            sa.red = x.red;
+            sa.n_prow = x.n_prow;
+            sa.nd = x.nd;
+            sa.g_base = 0;  // the launch's element index is the logical index
+            sa.s_base = x.s_shift;
+            sa.p_base = x.q_shift;
+            sa.j0 = p0;
+            sa.j1 = p1;
+            sa.c = x.c;
+            sa.cdev = x.cdev;
+            sa.ws_norm = x.ws_norm;
+            sa.ws_bad = x.ws_bad;
+            sa.ws_mode = x.ws_mode;
+            const zero_tma::Ring rg = zero_ring::ring_for_launch(ring, p1 - p0, x.nd, shapes.sms, shapes.tma_smem);
+            const uint64_t tiles = (p1 - p0 + rg.tile - 1) / rg.tile;
+            const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
+            peer_tma_kernel(rg.groups, rg.vw)<<<grid, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes,
+                                                 stream>>>(sa, rg, tab);
+        } else if (vec) {
+            k_step_peer<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
+        } else {
+            k_step_peer_scalar<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
+        }
         return check_launch("zero_step_peers kernel launch");
     };
     for (uint64_t bk = first; bk < first + count; ++bk) {

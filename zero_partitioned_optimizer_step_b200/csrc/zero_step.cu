@@ -45,6 +45,7 @@
 #include "zero_device.cuh"
 #include "zero_guard.cuh"
 #include "zero_tma.cuh"
+#include "zero_ring.cuh"
 #include "zero_host.cuh"
 #include "zero_internal.h"
 
@@ -52,10 +53,18 @@ using zero_detail::set_error;
 using zero_host::aligned16;
 using zero_host::check_launch;
 using zero_host::mult8;
+using zero_ring::choose_ring;
+using zero_ring::kernel_choice;
+using zero_ring::ring_for_launch;
 
 namespace {
 
 using namespace zero_dev;
+
+// The bulk-copy kernels' device error word on each device (1: a bounded
+// wait gave up; 2: a stage held another tile than expected).  Kernels get its
+// address in their Ring; zero_stream_status() reads and clears it.
+__device__ int g_wait_error;
 
 // K1, vector path: 8 elements (16 B of bf16, 32 B of fp32) per thread and
 // iteration.  Preconditions (checked on the host): j0, j1, all bases, strides,
@@ -228,16 +237,20 @@ __global__ void __launch_bounds__(kThreads) k_gather(const uint16_t *src, uint64
 
 // ----------------------------------------------------------------- host side
 
-// The bulk-copy kernel instantiations: owner map x consumer groups x vector width.
-using TmaKernel = void (*)(const StepArgs, const zero_tma::Ring);
+// The bulk-copy kernel instantiations: owner map x consumer groups x vector
+// width, for the fused step (rows = the Nd gradient rows) and for the guarded
+// step's second pass (row = the reduced gradient).
+template <int SRC>
+using TmaKernelOf = void (*)(const StepArgs, const zero_tma::Ring, const typename zero_tma::ExtraOf<SRC>::type);
+using TmaKernel = TmaKernelOf<zero_tma::kGradRows>;
+using ApplyKernel = TmaKernelOf<zero_tma::kReduced>;
 
-template <bool OM>
-TmaKernel tma_kernel(uint32_t groups, uint32_t vw) {
+template <bool OM, int SRC = zero_tma::kGradRows>
+TmaKernelOf<SRC> tma_kernel(uint32_t groups, uint32_t vw) {
+    using namespace zero_tma;
     if (groups == 2)
-        return vw == 2 ? zero_tma::k_step_tma<OM, 2, 2>
-                       : (vw == 4 ? zero_tma::k_step_tma<OM, 2, 4> : zero_tma::k_step_tma<OM, 2, 8>);
-    return vw == 2 ? zero_tma::k_step_tma<OM, 1, 2>
-                   : (vw == 4 ? zero_tma::k_step_tma<OM, 1, 4> : zero_tma::k_step_tma<OM, 1, 8>);
+        return vw == 2 ? k_step_tma<OM, 2, 2, SRC> : (vw == 4 ? k_step_tma<OM, 2, 4, SRC> : k_step_tma<OM, 2, 8, SRC>);
+    return vw == 2 ? k_step_tma<OM, 1, 2, SRC> : (vw == 4 ? k_step_tma<OM, 1, 4, SRC> : k_step_tma<OM, 1, 8, SRC>);
 }
 
 // Launch shapes of the step kernels on one device, computed once per device:
@@ -246,6 +259,7 @@ TmaKernel tma_kernel(uint32_t groups, uint32_t vw) {
 // (one CTA per SM: its ring takes most of shared memory), and the dynamic
 // shared memory the bulk-copy kernel may use.
 struct DeviceShapes {
+    int *err = nullptr;       // g_wait_error on this device
     uint32_t grid_ldg = 0;
     uint32_t grid_guard = 0;  // the guarded step's two passes (fewer registers)
     uint32_t sms = 0;
@@ -276,6 +290,9 @@ zero_status_t device_shapes(DeviceShapes *out) {
     cudaFuncAttributes fa{};
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
     DeviceShapes d;
+    void *err = nullptr;
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&err, g_wait_error);
+    d.err = static_cast<int *>(err);
     d.sms = uint32_t(std::max(1, sms));
     d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
     d.grid_guard = std::min(uint32_t(std::max(1, sms) * std::max(1, std::min(occ_r, occ_a))), zero_detail::kMaxSlots);
@@ -283,145 +300,20 @@ zero_status_t device_shapes(DeviceShapes *out) {
     d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
     if (d.tma_smem > 0) {
         for (uint32_t g : {1u, 2u})
-            for (uint32_t vw : {2u, 4u, 8u})
-                for (TmaKernel f : {tma_kernel<true>(g, vw), tma_kernel<false>(g, vw)})
+            for (uint32_t vw : {2u, 4u, 8u}) {
+                const void *fs[] = {reinterpret_cast<const void *>(tma_kernel<true>(g, vw)),
+                                    reinterpret_cast<const void *>(tma_kernel<false>(g, vw)),
+                                    reinterpret_cast<const void *>(tma_kernel<true, zero_tma::kReduced>(g, vw)),
+                                    reinterpret_cast<const void *>(tma_kernel<false, zero_tma::kReduced>(g, vw))};
+                for (const void *f : fs)
                     if (e == cudaSuccess)
-                        e = cudaFuncSetAttribute(reinterpret_cast<const void *>(f),
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
+                        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
+            }
     }
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("device query: ") + cudaGetErrorString(e));
     cache[dev] = d;
     *out = d;
     return ZERO_OK;
-}
-
-uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127)); }
-
-// Shared-memory ring of the bulk-copy kernel for Nd gradient rows.  Each
-// tile pays a fixed synchronisation latency, so tiles are large; two consumer
-// groups help where a tile is cheap to compute.  Shapes measured best on B200
-// at 64 MB buckets (5e8 params), as (groups, tile, stages, elements/thread):
-//   Nd <= 2: (2, 2048, 4, 8)     Nd <= 4: (1, 4096, 2, 8)     Nd <= 8: (1, 2048, 3, 8)
-//   Nd <= 16: (1, 1024, 4, 4)    Nd <= 32: (1, 1024, 2, 8)
-//   Nd <= 64: (1, 512, 3, 4)
-// Read-heavy steps (parameters written once: stage 3 or one owner) do better
-// with larger bulk copies, i.e. larger tiles: Nd <= 16 takes (1, 2048, 2, 8)
-// (the stage-3 1.3B workload at Nd = 16).  Beyond 64 ranks the 16-byte-load
-// kernel is used, and also for read-heavy steps with more than 32 ranks: there
-// every gradient row of a 512-element tile is a 1 KB bulk copy, and the rate
-// at which an SM completes such copies caps the read bandwidth (0.64 of copy
-// bandwidth against 0.80 for the load kernel, one owner of 64 ranks).  With
-// two groups the stage count is even (each group owns half the stages).
-// ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS / ZERO_TMA_VW override the
-// shape (tuning; a tile must be a positive multiple of 256).
-zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t groups) {
-    zero_tma::Ring q;
-    q.tile = uint32_t(t);
-    q.off_w = align128(uint64_t(nd) * t * 2);
-    q.off_m = q.off_w + align128(4 * t);
-    q.off_v = q.off_m + align128(4 * t);
-    q.stage_bytes = q.off_v + align128(4 * t);
-    q.stages = stages;
-    q.groups = groups;
-    return q;
-}
-
-bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, zero_tma::Ring *r) {
-    long force_t = 0, force_s = 0, force_g = 0, force_v = 0;
-    if (const char *e = std::getenv("ZERO_TMA_TILE")) force_t = std::strtol(e, nullptr, 10);
-    if (const char *e = std::getenv("ZERO_TMA_STAGES")) force_s = std::strtol(e, nullptr, 10);
-    if (const char *e = std::getenv("ZERO_TMA_GROUPS")) force_g = std::strtol(e, nullptr, 10);
-    if (const char *e = std::getenv("ZERO_TMA_VW")) force_v = std::strtol(e, nullptr, 10);
-    uint32_t groups, stages, vw;
-    uint64_t tile;
-    if (force_t >= 256 && force_t % 256 == 0 && force_t <= 16384) {
-        tile = uint64_t(force_t);
-        groups = force_g == 2 ? 2 : 1;
-        stages = force_s >= 2 ? uint32_t(std::min<long>(force_s, zero_tma::kMaxStages)) : zero_tma::kMaxStages;
-        const uint64_t busy = tile * groups / zero_tma::kConsumers;  // keep a group's threads busy
-        vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
-    } else if (nd <= 2) {
-        groups = 2, tile = 2048, stages = 4, vw = 8;
-    } else if (nd <= 4) {
-        groups = 1, tile = 4096, stages = 2, vw = 8;
-    } else if (nd <= 8) {
-        groups = 1, tile = 2048, stages = 3, vw = 8;
-    } else if (nd <= 16 && read_heavy) {
-        groups = 1, tile = 2048, stages = 2, vw = 8;
-    } else if (nd <= 16) {
-        groups = 1, tile = 1024, stages = 4, vw = 4;
-    } else if (nd <= 32) {
-        groups = 1, tile = 1024, stages = 2, vw = 8;
-    } else if (nd <= 64 && !read_heavy) {
-        groups = 1, tile = 512, stages = 3, vw = 4;
-    } else {
-        return false;
-    }
-    if (force_v == 2 || force_v == 4 || force_v == 8) vw = uint32_t(force_v);
-    zero_tma::Ring q = ring_for(nd, tile, 0, groups);
-    q.vw = vw;
-    // ZERO_TEST_STALL_PRODUCER=<cta>: that CTA's producer issues nothing, so
-    // its consumers' bounded waits run out (tests the ZERO_ETIMEOUT path)
-    q.stall_cta = 0xffffffffu;
-    if (const char *e = std::getenv("ZERO_TEST_STALL_PRODUCER")) {
-        char *end = nullptr;
-        const unsigned long v = std::strtoul(e, &end, 10);
-        if (end != e && v < 0xffffffffu) q.stall_cta = uint32_t(v);
-    }
-    uint64_t ns = std::min<uint64_t>(budget / q.stage_bytes, stages);
-    ns -= ns % groups;  // every stage belongs to one group
-    if (ns < 2) return false;
-    q.stages = uint32_t(ns);
-    *r = q;
-    return true;
-}
-
-// A small bucket is over soon after a CTA's ring has filled, and the next
-// bucket's CTAs (launched early through programmatic dependent launch) cannot
-// start on an SM while this ring takes most of its shared memory.  Below
-// 32 x 2048 elements per SM the ring is cut to half of the SM's shared memory (tile
-// halved while needed, at least 512, and as many stages as then fit), so two
-// CTAs share an SM and the next bucket's loads overlap this one's tail.
-// Measured on B200 (5e8 params): +50 % at 1-2 MB buckets for Nd <= 8 and
-// +10-20 % up to 16 MB; from 32 MB up the full ring is faster.
-// ZERO_TMA_ADAPT=0, or a forced ZERO_TMA_TILE, keeps the chosen ring;
-// ZERO_TMA_ADAPT_TILES=<n> moves the threshold to n x 2048 elements per SM
-// (tuning).
-zero_tma::Ring ring_for_launch(const zero_tma::Ring &r, uint64_t n, uint32_t nd, uint32_t sms,
-                               uint32_t budget) {
-    static const bool off = [] {
-        const char *e = std::getenv("ZERO_TMA_ADAPT");
-        return (e && e[0] == '0') || std::getenv("ZERO_TMA_TILE") != nullptr;
-    }();
-    static const uint64_t per_sm = [] {
-        const char *e = std::getenv("ZERO_TMA_ADAPT_TILES");
-        const long v = e ? std::strtol(e, nullptr, 10) : 0;
-        return uint64_t(v > 0 ? v : 32);
-    }();
-    if (off || n >= 2048ull * per_sm * sms) return r;
-    const uint64_t half = budget / 2 - 1024;  // room for a second CTA's ring and static shared memory
-    for (uint64_t tile = r.tile; tile >= 512; tile /= 2) {
-        zero_tma::Ring q = ring_for(nd, tile, 0, r.groups);
-        uint64_t ns = std::min<uint64_t>(half / q.stage_bytes, zero_tma::kMaxStages);
-        ns -= ns % r.groups;
-        if (ns < 2 || ns < r.groups * 2) continue;
-        q.stall_cta = r.stall_cta;
-        const uint64_t busy = tile * r.groups / zero_tma::kConsumers;
-        q.vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
-        q.stages = uint32_t(ns);
-        return q;
-    }
-    return r;
-}
-
-// ZERO_STEP_KERNEL=ldg|tma picks the vector kernel for aligned bucket bodies
-// (default: the bulk-copy kernel whenever its ring fits).
-int kernel_choice() {
-    const char *s = std::getenv("ZERO_STEP_KERNEL");
-    if (!s) return 0;
-    if (std::strcmp(s, "ldg") == 0) return 1;
-    if (std::strcmp(s, "tma") == 0) return 2;
-    return 0;
 }
 
 AdamConsts make_consts(const zero_adam_t &a, uint64_t t) {
@@ -499,7 +391,7 @@ struct Launcher {
                 const size_t smem = size_t(rg.stages) * rg.stage_bytes;
                 TmaKernel f = owner_map ? tma_kernel<true>(rg.groups, rg.vw)
                                         : tma_kernel<false>(rg.groups, rg.vw);
-                launch_ex(f, grid, zero_tma::kThreads, smem, stream, dep, b, rg);
+                launch_ex(f, grid, zero_tma::kThreads, smem, stream, dep, b, rg, zero_tma::NoExtra{});
             } else if (vec) {
                 const bool rb8 = ldg_rows(b.nd) == 8;
                 auto f = owner_map ? (rb8 ? k_step_vec8<true, 8, kMinB> : k_step_vec8<true, kRB, kMinB>)
@@ -653,8 +545,8 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
     L.want_ws = b->grad_norm_sq || b->overflow;
     L.pdl = pdl_enabled();
     const int choice = kernel_choice();
-    L.use_tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, &L.ring)
-                            : choice != 1 && choose_ring(p->nd, a.n_prow == 1, shapes.tma_smem, &L.ring);
+    L.use_tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, shapes.err, &L.ring)
+                            : choice != 1 && choose_ring(p->nd, a.n_prow == 1, shapes.tma_smem, shapes.err, &L.ring);
     if (L.want_ws && first == 0) {
         // the step's first call zeroes the per-CTA norm slots
         cudaError_t e = cudaMemsetAsync(b->workspace, 0, zero_detail::kWorkspaceBytes, L.stream);
@@ -720,16 +612,23 @@ ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const vo
     return ZERO_OK;
 }
 
+zero_status_t zero_detail::wait_error_word(int **out) {
+    DeviceShapes shapes;
+    zero_status_t st = device_shapes(&shapes);
+    if (st == ZERO_OK) *out = shapes.err;
+    return st;
+}
+
 ZERO_API zero_status_t zero_stream_status(void *stream) {
     zero_detail::clear_error();
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("zero_stream_status: ") + cudaGetErrorString(e));
     int v = 0;
-    e = cudaMemcpyFromSymbol(&v, zero_tma::g_wait_error, sizeof v);
+    e = cudaMemcpyFromSymbol(&v, g_wait_error, sizeof v);
     if (e != cudaSuccess) return set_error(ZERO_ECUDA, std::string("zero_stream_status: ") + cudaGetErrorString(e));
     if (v) {
         const int zero = 0;
-        cudaMemcpyToSymbol(zero_tma::g_wait_error, &zero, sizeof zero);
+        cudaMemcpyToSymbol(g_wait_error, &zero, sizeof zero);
         return set_error(ZERO_ETIMEOUT,
                          v == 2 ? "zero_stream_status: the bulk-copy step kernel found a stage holding the wrong "
                                   "tile and gave up; the outputs of the steps since the last check are not valid"
@@ -750,9 +649,9 @@ ZERO_API zero_status_t zero_step_kernel(const zero_plan_t *p, int32_t owner_view
     const bool replicas = owner_view < 0 && p->stage <= 2;
     zero_tma::Ring ring{};
     const int choice = kernel_choice();
-    const bool tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, &ring)
+    const bool tma = choice == 2 ? choose_ring(p->nd, false, shapes.tma_smem, shapes.err, &ring)
                                  : choice != 1 && choose_ring(p->nd, !replicas || p->nd == 1,
-                                                              shapes.tma_smem, &ring);
+                                                              shapes.tma_smem, shapes.err, &ring);
     *kind = tma ? ZERO_KERNEL_BULK_COPY : ZERO_KERNEL_VECTOR_LOAD;
     return ZERO_OK;
 }
@@ -813,7 +712,19 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
                                                              guard->skip_nonfinite ? 1 : 0);
     st = check_launch("zero_step_guarded finalize launch");
     if (st != ZERO_OK) return st;
-    // pass 2: Adam from the reduced gradients (no-op when the step is skipped)
+    // pass 2: Adam from the reduced gradients (no-op when the step is skipped).
+    // When the parameters are written once (stage 3), aligned bodies run in
+    // the bulk-copy kernel with the reduced gradient as its one fp32 row (a
+    // ring shaped as for two bf16 rows): 0.95 of copy bandwidth against 0.91
+    // for k_apply on the stage-3 1.3B workload.  With Nd replicas to write
+    // (28 B of stores per element at Nd = 8) k_apply with 32-byte accesses is
+    // faster (189 us against 200 us per 25M-element bucket).
+    // ZERO_STEP_KERNEL=tma|ldg forces either.
+    zero_tma::Ring ring{};
+    const int choice = kernel_choice();
+    const bool tma = (choice == 2 || (choice == 0 && a.n_prow == 1)) &&
+                     choose_ring(2, false, shapes.tma_smem, shapes.err, &ring);
+    a.ws_mode = 0;
     for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
         StepArgs x;
         bool om, vec_ok;
@@ -822,7 +733,15 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             StepArgs y = x;
             y.j0 = j0;
             y.j1 = j1;
-            if (vec && om && w32) zero_guarded::k_apply<8, true, true><<<grid, kThreads, 0, stream>>>(y, gw);
+            if (vec && tma) {
+                const zero_tma::Ring rg = ring_for_launch(ring, j1 - j0, 2, shapes.sms, shapes.tma_smem);
+                const uint64_t tiles = (j1 - j0 + rg.tile - 1) / rg.tile;
+                const uint32_t g = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
+                ApplyKernel f = om ? tma_kernel<true, zero_tma::kReduced>(rg.groups, rg.vw)
+                                   : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw);
+                f<<<g, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes, stream>>>(y, rg,
+                                                                                      zero_tma::ApplyExtra{gw});
+            } else if (vec && om && w32) zero_guarded::k_apply<8, true, true><<<grid, kThreads, 0, stream>>>(y, gw);
             else if (vec && w32) zero_guarded::k_apply<8, false, true><<<grid, kThreads, 0, stream>>>(y, gw);
             else if (vec && om) zero_guarded::k_apply<8, true><<<grid, kThreads, 0, stream>>>(y, gw);
             else if (vec) zero_guarded::k_apply<8, false><<<grid, kThreads, 0, stream>>>(y, gw);

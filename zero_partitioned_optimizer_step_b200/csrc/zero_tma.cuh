@@ -14,11 +14,12 @@
 // bytes in flight.  No multicast is used.
 //
 // Every wait is bounded (kWaitLimitNs of %globaltimer).  A thread that gives
-// up sets the CTA's abort flag and the device error word g_wait_error; the
+// up sets the CTA's abort flag and the device error word; the
 // consumers leave the loop together (the decision is an OR-reduction over a
 // barrier, so no consumer is left alone at a barrier), the producer waits a
 // bounded time for the loads it issued, and the kernel returns.
-// zero_stream_status() reports the error word.
+// zero_stream_status() reports the error word (one word per device, owned by
+// the library; its address travels in the Ring).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -49,6 +50,9 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 // `tile` bf16 at offset 0, then w, m, v (fp32).  `vw` is the per-thread
 // vector width the kernel was instantiated with.
 struct Ring {
+    int *err;            // device error word: 1 once a bounded wait has given up,
+                         // 2 if a consumer found a stage holding another tile
+                         // than the one it expected
     uint32_t stall_cta;  // test of the bounded waits: this CTA's producer issues
                          // nothing (0xffffffff: none)
     uint32_t vw;
@@ -58,10 +62,6 @@ struct Ring {
     uint32_t stage_bytes;
     uint32_t off_w, off_m, off_v;
 };
-
-// Device error word: 1 once a bounded wait has given up, 2 if a consumer found
-// a stage holding another tile than the one it expected.
-__device__ int g_wait_error;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -104,8 +104,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 // Wait for the phase of `bar` with the given parity.  Gives up (returning
 // false) when the CTA's abort flag is raised, or after kWaitLimitNs, in which
-// case it raises the abort flag and the device error word.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// case it raises the abort flag and sets the device error word *err to 1.
+static __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                              int *err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
@@ -114,7 +115,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 *abort_flag = 1;
-                atomicExch(&g_wait_error, 1);
+                atomicExch(err, 1);
                 return false;
             }
         }
@@ -229,8 +230,55 @@ __device__ __forceinline__ void stg_bf16_rows(uint16_t *p, const float w[VW], ui
     }
 }
 
-template <bool OWNER_MAP, int GROUPS, int VW>
-__global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, const Ring ring) {
+// Where a tile's rows come from, and where the parameters go.
+//   kGradRows: the Nd bf16 gradient rows at a.grads + r * a.grad_stride
+//              (the fused step), parameters at a.params (+ row * param_stride);
+//   kReduced:  one fp32 row, the reduced gradient at a.red in state order, and
+//              g = (g_sum * grad_scale) * coef from the guarded step's decision,
+//              nothing at all if that decision is to skip (its second pass);
+//   kPeerRows: the Nd bf16 gradient rows at x.g[r] and the parameter rows at
+//              x.p[q]: other ranks' buffers reached through their pointers.
+enum RowSource { kGradRows = 0, kReduced = 1, kPeerRows = 2 };
+
+struct NoExtra {};
+struct ApplyExtra {
+    const zero_dev::GuardWord *gw;
+};
+
+template <int SRC>
+struct ExtraOf {
+    using type = NoExtra;
+};
+template <>
+struct ExtraOf<kReduced> {
+    using type = ApplyExtra;
+};
+template <>
+struct ExtraOf<kPeerRows> {
+    using type = zero_dev::PeerTable;
+};
+
+// bf16(w) of VW elements to `rows` parameter rows given by pointer
+template <int VW>
+__device__ __forceinline__ void stg_bf16_ptrs(uint16_t *const *rows, uint64_t off, const float w[VW], uint32_t n) {
+    uint32_t pk[VW / 2];
+#pragma unroll
+    for (int h = 0; h < VW / 2; ++h) pk[h] = zero_dev::pack_bf16x2(w[2 * h], w[2 * h + 1]);
+    for (uint32_t r = 0; r < n; ++r) {
+        uint16_t *q = rows[r] + off;
+        if constexpr (VW == 2) {
+            __stcs(reinterpret_cast<unsigned int *>(q), pk[0]);
+        } else if constexpr (VW == 4) {
+            __stcs(reinterpret_cast<uint2 *>(q), make_uint2(pk[0], pk[1]));
+        } else {
+            __stcs(reinterpret_cast<uint4 *>(q), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        }
+    }
+}
+
+template <bool OWNER_MAP, int GROUPS, int VW, int SRC = kGradRows>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_step_tma(const StepArgs a, const Ring ring, const typename ExtraOf<SRC>::type x) {
     constexpr uint32_t kGroupThreads = kConsumers / GROUPS;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
@@ -239,11 +287,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
     __shared__ int s_abort;
     __shared__ double s_norm[kConsumerWarps];
     __shared__ uint32_t s_bad[kConsumerWarps];
+    __shared__ const uint16_t *s_rows[SRC == kPeerRows ? zero_dev::kMaxPeers : 1];
+    __shared__ uint16_t *s_prow[SRC == kPeerRows ? zero_dev::kMaxPeers : 1];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t T = ring.tile;
     const uint32_t NS = ring.stages;
     const uint64_t n_tiles = (a.j1 - a.j0 + T - 1) / T;
+    float coef = 1.0f;
+    if constexpr (SRC == kReduced) {
+        const zero_dev::GuardWord g = *x.gw;
+        if (g.skip) return;  // every thread, before any barrier
+        coef = g.coef;
+    }
 
     zero_dev::pdl_launch_dependents();
     if (threadIdx.x == 0) {
@@ -254,18 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
         s_abort = 0;
         fence_barrier_init();
     }
+    if constexpr (SRC == kPeerRows) {
+        for (uint32_t i = threadIdx.x; i < a.nd; i += kThreads) s_rows[i] = x.g[i];
+        for (uint32_t i = threadIdx.x; i < a.n_prow; i += kThreads) s_prow[i] = x.p[i];
+    }
     __syncthreads();
     volatile int *abort_flag = &s_abort;
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
         if (blockIdx.x == ring.stall_cta) return;  // consumers' waits run out
+        constexpr uint32_t kRowBytes = SRC == kReduced ? 4u : 0u;
         uint32_t k = 0;
         for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++k) {
             const uint32_t s = k % NS;
             if (k >= NS) {
                 int ok = 1;
-                if (lane == 0) ok = mbar_wait(&empty_bar[s], ((k / NS) - 1) & 1u, abort_flag);
+                if (lane == 0) ok = mbar_wait(&empty_bar[s], ((k / NS) - 1) & 1u, abort_flag, ring.err);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
@@ -275,16 +336,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
             unsigned char *st = smem + size_t(s) * ring.stage_bytes;
             if (lane == 0) {
                 stage_tile[s] = tile;  // published by the arrive below (release)
-                mbar_arrive_expect_tx(&full_bar[s], n * (2u * a.nd + 12u));
+                const uint32_t per = SRC == kReduced ? 4u + 12u : 2u * a.nd + 12u;
+                mbar_arrive_expect_tx(&full_bar[s], n * per);
             }
             __syncwarp();
-            const uint16_t *g = a.grads + uint64_t(a.g_base + int64_t(jb));
-            for (uint32_t r = lane; r < a.nd; r += 32)
-                bulk_load(st + size_t(r) * T * 2, g + uint64_t(r) * a.grad_stride, n * 2u, &full_bar[s]);
+            if constexpr (SRC != kReduced) {
+                const int64_t gofs = a.g_base + int64_t(jb);
+                for (uint32_t r = lane; r < a.nd; r += 32) {
+                    const uint16_t *src = SRC == kPeerRows ? s_rows[r] + gofs
+                                                           : a.grads + uint64_t(gofs) + uint64_t(r) * a.grad_stride;
+                    bulk_load(st + size_t(r) * T * 2, src, n * 2u, &full_bar[s]);
+                }
+            }
             if (lane == 0) {
                 for_each_segment<OWNER_MAP>(a, jb, je, [&](uint64_t js, uint64_t cnt, uint64_t so, uint64_t) {
                     const uint64_t off = js - jb;
                     const uint64_t si = uint64_t(a.s_base + int64_t(js)) + so;
+                    if (kRowBytes) bulk_load(st + off * 4, a.red + si, uint32_t(cnt * 4), &full_bar[s]);
                     bulk_load(st + ring.off_w + off * 4, a.w + si, uint32_t(cnt * 4), &full_bar[s]);
                     bulk_load(st + ring.off_m + off * 4, a.m + si, uint32_t(cnt * 4), &full_bar[s]);
                     bulk_load(st + ring.off_v + off * 4, a.v + si, uint32_t(cnt * 4), &full_bar[s]);
@@ -297,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
             volatile int *never = &dummy;
             for (uint32_t i = 0; i < NS && i < k; ++i) {
                 const uint32_t kk = k - 1 - i;
-                mbar_wait(&full_bar[kk % NS], (kk / NS) & 1u, never);
+                mbar_wait(&full_bar[kk % NS], (kk / NS) & 1u, never, ring.err);
             }
         }
         return;
@@ -316,11 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
     for (uint64_t tile = blockIdx.x + uint64_t(grp) * gridDim.x; tile < n_tiles;
          tile += uint64_t(GROUPS) * gridDim.x, k += GROUPS) {
         const uint32_t s = k % NS;
-        bool failed = !mbar_wait(&full_bar[s], (k / NS) & 1u, abort_flag);
+        bool failed = !mbar_wait(&full_bar[s], (k / NS) & 1u, abort_flag, ring.err);
         if (!failed && stage_tile[s] != tile) {  // self-check of the ring protocol
             failed = true;
             *abort_flag = 1;
-            atomicExch(&g_wait_error, 2);
+            atomicExch(ring.err, 2);
         }
         const uint64_t jb = a.j0 + tile * T;
         const uint32_t n = uint32_t(min(jb + T, a.j1) - jb);
@@ -328,14 +396,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
         if (!failed) {
             const uint32_t nv = n / VW;
             for (uint32_t vv = gt; vv < nv; vv += kGroupThreads) {
-                const unsigned char *gp = st + size_t(vv) * (2 * VW);
-                float sum[VW], f[VW];
-                lds_bf16<VW>(gp, sum);
+                float sum[VW];
+                if constexpr (SRC == kReduced) {
+                    lds_f32<VW>(st + size_t(vv) * (4 * VW), sum);
+                } else {
+                    const unsigned char *gp = st + size_t(vv) * (2 * VW);
+                    float f[VW];
+                    lds_bf16<VW>(gp, sum);
 #pragma unroll 4
-                for (uint32_t r = 1; r < a.nd; ++r) {
-                    lds_bf16<VW>(gp + size_t(r) * T * 2, f);
+                    for (uint32_t r = 1; r < a.nd; ++r) {
+                        lds_bf16<VW>(gp + size_t(r) * T * 2, f);
 #pragma unroll
-                    for (int e = 0; e < VW; ++e) sum[e] = __fadd_rn(sum[e], f[e]);
+                        for (int e = 0; e < VW; ++e) sum[e] = __fadd_rn(sum[e], f[e]);
+                    }
                 }
                 float wv[VW], mv[VW], vq[VW];
                 lds_f32<VW>(st + ring.off_w + size_t(vv) * (4 * VW), wv);
@@ -352,13 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
                 const uint64_t o = OWNER_MAP ? j / a.shard : 0;
                 const uint64_t si = uint64_t(a.s_base + int64_t(j)) + o * a.jump;
                 const uint64_t pi = uint64_t(a.p_base + int64_t(j)) + o * a.p_jump;
-                if (a.red) stg_f32<VW>(a.red + si, sum);
+                if (SRC != kReduced && a.red) stg_f32<VW>(a.red + si, sum);
 #pragma unroll
-                for (int e = 0; e < VW; ++e) zero_dev::adam1(sum[e], C, wv[e], mv[e], vq[e]);
+                for (int e = 0; e < VW; ++e) zero_dev::adam1c(sum[e], coef, C, wv[e], mv[e], vq[e]);
                 stg_f32<VW>(a.w + si, wv);
                 stg_f32<VW>(a.m + si, mv);
                 stg_f32<VW>(a.v + si, vq);
-                stg_bf16_rows<VW>(a.params + pi, wv, a.n_prow, a.param_stride);
+                if constexpr (SRC == kPeerRows) stg_bf16_ptrs<VW>(s_prow, pi, wv, a.n_prow);
+                else stg_bf16_rows<VW>(a.params + pi, wv, a.n_prow, a.param_stride);
             }
         }
         // the whole group has read the stage (or the CTA is giving up): same
@@ -367,6 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_step_tma(const StepArgs a, cons
         if (gt == 0) mbar_arrive(&empty_bar[s]);
     }
 
+    if constexpr (SRC == kPeerRows) {
+        // every consumer's peer stores are performed before the kernel
+        // completes: a consumer barrier, then one cumulative system fence
+        barrier_or(1 + GROUPS, kConsumers, false);
+        if (ct == 0) __threadfence_system();
+    }
     zero_dev::pdl_wait();  // predecessor done: its norm slots are final
     if (a.ws_mode) {
 #pragma unroll
