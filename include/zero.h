@@ -13,6 +13,8 @@
  *      replica (stages 0-2), or to the owner's shard only (stage 3), from
  *      where zero_gather_layer() materialises one layer at a time.
  * All of it runs in hand-written CUDA kernels; there is no CPU path.
+ * zero_step_peers() runs one rank's share of the same step when the ranks
+ * have their own buffers (one GPU per rank; see "Ranks as devices" below).
  *
  * Sources (three web pages about ZeRO, arXiv 1910.02054):
  *  [MM] mind-map page "ZeRO 真正在做什么：长期分开存，计算时临时拼齐"
