@@ -225,3 +225,32 @@ def test_reshard_argument_checks_on_host():
     assert L.zero_reshard(a.handle, None, b.handle, ctypes.c_void_p(8192), 4, None) == Z.ZERO_EINVAL
     assert L.zero_reshard(a.handle, ctypes.c_void_p(4098), b.handle, ctypes.c_void_p(8192), 4,
                           None) == Z.ZERO_EINVAL
+
+
+def test_plain_c_caller(tmp_path):
+    """A C program (tests/c/plan_example.c) compiled against include/zero.h
+    and linked to libzero.so gets the oracle's plan through the C ABI."""
+    lib_dir = os.path.dirname(Z.LIB_PATH)
+    exe = tmp_path / "plan_example"
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-O1", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "plan_example.c"), "-L", lib_dir, "-lzero",
+                    "-Wl,-rpath," + lib_dir, "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout
+    got = {}
+    for line in out.splitlines():
+        k, v = line.split(" ", 1)
+        got[k] = v
+    op = OP.make_plan(124_439_808, 8, 2, 25_000_000)
+    assert int(got["gpt2.psi_pad"]) == op.psi_pad and int(got["gpt2.S"]) == op.S
+    assert int(got["gpt2.n_buckets"]) == len(op.buckets)
+    assert int(got["gpt2.comm_elems"]) == OP.comm_elems_per_rank(op)
+    assert int(got["gpt2.hbm_step"]) == OP.hbm_step_bytes(op, False, False)
+    for st in range(4):
+        assert int(got["gpt2.mem_stage%d" % st]) == OP.memory_bytes_per_rank_padded(op, st)
+    assert int(got["gpt2.owner_of_77777777"]) == OP.locate(op, 77_777_777)[1]
+    o3 = OP.make_plan(350_008, 5, 3, 65_536, align=8, unit_elems=[100_000, 7, 250_001])
+    for u in range(3):
+        assert got["st3.unit%d" % u] == "%d %d %d" % (o3.unit_pad[u], o3.unit_shard[u], o3.unit_offset[u])
+    assert got["st3.release_unheld"] == "%d ESTATE" % Z.ZERO_ESTATE
+    assert got["abi"] == "3"

@@ -231,3 +231,55 @@ def test_peer_step_maps_every_other_rank_and_unmaps_on_close():
         assert [g[o] for o in others] == [1000 * (2 * i + 1) for i in range(len(others))]
         assert [p[o] for o in others] == [1000 * (2 * i + 2) for i in range(len(others))]
         assert sorted(closed) == sorted([g[o] for o in others] + [p[o] for o in others])
+
+
+def _dropout_worker(rank, world, port, out):
+    """Rank 1 builds its PeerStep and then leaves without stepping; rank 0's
+    step must end with an error from the process group's timeout, not hang."""
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import zero_partitioned_optimizer_step_b200 as Zw
+    from zero_partitioned_optimizer_step_b200.peer import PeerStep
+    store = dist.TCPStore("127.0.0.1", port, world, rank == 0, timeout=datetime.timedelta(seconds=30))
+    dist.init_process_group("gloo", store=store, rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=3))
+
+    class Buf:
+        def __init__(self, tag):
+            self.tag, self.device = tag, "cpu"
+
+    calls = []
+    plan = Zw.zero_plan(1000, world, 2, 100)
+    ps = PeerStep(plan, Buf("g"), Buf("p"), None, None, None, ipc_open=lambda h: 4096,
+                  ipc_close=lambda p: None, ipc_export=lambda t: b"x")
+    if rank == 1:
+        out.put((rank, "left"))
+        out.close()
+        out.join_thread()   # the message is out before the process is
+        os._exit(0)   # gone between steps: no kernel or collective of it in flight
+    import zero_partitioned_optimizer_step_b200.peer as P
+    P.zero_step_peers = lambda *a, **k: calls.append("kernel")   # the barrier decides
+    try:
+        ps.step(dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, grad_scale=0.5), 1)
+        out.put((rank, "stepped"))
+    except Exception as e:  # the expected path
+        out.put((rank, "error:" + type(e).__name__ + ":" + ("kernel" if calls else "no-kernel")))
+
+
+def test_a_rank_that_leaves_makes_the_next_step_fail_not_hang():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dropout_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = dict(q.get(timeout=120) for _ in procs)
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.exitcode is None:
+                p.kill()
+    assert res[1] == "left"
+    assert res[0].startswith("error:") and res[0].endswith(":no-kernel"), res
