@@ -38,6 +38,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -94,6 +95,7 @@ __device__ __forceinline__ void cta_release_system() {
 // adds.  Preconditions (host): p0, p1, s_shift, q_shift multiples of 8 and
 // every pointer 16-byte aligned.
 __global__ void __launch_bounds__(kThreads, kPeerMinB) k_step_peer(const PeerArgs a, const PeerTable T) {
+    pdl_launch_dependents();
     __shared__ const uint16_t *sg[kMaxPeers];
     __shared__ uint16_t *sp[kMaxPeers];
     for (uint32_t i = threadIdx.x; i < a.nd; i += kThreads) sg[i] = T.g[i];
@@ -162,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, kPeerMinB) k_step_peer(const PeerArg
         for (uint32_t q = 0; q < a.n_prow; ++q) __stcs(reinterpret_cast<uint4 *>(sp[q] + pi), pk);
     }
     cta_release_system();
+    pdl_wait();  // predecessor done: its norm slots are final
     if (a.ws_mode) block_partials(acc, bad, a.ws_norm, a.ws_bad);
 }
 
@@ -288,6 +291,23 @@ zero_status_t peer_shapes(PeerShapes *out) {
     return ZERO_OK;
 }
 
+// Launch with or without programmatic dependent launch on the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), uint32_t grid, uint32_t block, size_t smem,
+                       cudaStream_t stream, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 zero_status_t validate_peers(const zero_plan_t *p, const zero_peer_bufs_t *b, const zero_adam_t *adam,
                              uint64_t t) {
     if (!p || !b || !adam) return set_error(ZERO_EINVAL, "zero_step_peers: NULL argument");
@@ -393,11 +413,19 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
     if (st != ZERO_OK) return st;
     const bool tma = zero_ring::kernel_choice() == 2 &&
                      zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring);
+    // Vector launches after the first of the call overlap their predecessor
+    // (programmatic dependent launch): consecutive launches of one call share
+    // only the norm slots, which every kernel adds to after its predecessor
+    // has completed.  ZERO_PDL=0 turns it off.
+    const char *pdl_env = std::getenv("ZERO_PDL");
+    const bool pdl = !(pdl_env && pdl_env[0] == '0');
+    uint32_t launches = 0;
     auto launch = [&](uint64_t p0, uint64_t p1, bool vec) -> zero_status_t {
         if (p0 >= p1) return ZERO_OK;
         PeerArgs x = a;
         x.p0 = p0;
         x.p1 = p1;
+        const bool dep = pdl && launches++ > 0;
         if (vec && tma) {
             StepArgs sa{};
             sa.w = x.w;
@@ -419,10 +447,10 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
             const zero_tma::Ring rg = zero_ring::ring_for_launch(ring, p1 - p0, x.nd, shapes.sms, shapes.tma_smem);
             const uint64_t tiles = (p1 - p0 + rg.tile - 1) / rg.tile;
             const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
-            peer_tma_kernel(rg.groups, rg.vw)<<<grid, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes,
-                                                 stream>>>(sa, rg, tab);
+            launch_pdl(peer_tma_kernel(rg.groups, rg.vw), grid, zero_tma::kThreads,
+                       size_t(rg.stages) * rg.stage_bytes, stream, dep, sa, rg, tab);
         } else if (vec) {
-            k_step_peer<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
+            launch_pdl(k_step_peer, shapes.grid, kThreads, 0, stream, dep, x, tab);
         } else {
             k_step_peer_scalar<<<shapes.grid, kThreads, 0, stream>>>(x, tab);
         }
