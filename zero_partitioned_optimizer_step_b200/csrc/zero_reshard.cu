@@ -7,6 +7,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 
 #include "zero_device.cuh"
 #include "zero_host.cuh"
@@ -45,6 +46,7 @@ template <typename T> struct Vec<T, 1> { using type = T; };
 template <typename T, int V, int R>
 __global__ void __launch_bounds__(kThreads) k_reshard(const T *__restrict__ src, T *__restrict__ dst,
                                                      const ReshardArgs a) {
+    zero_dev::pdl_launch_dependents();
     using VT = typename Vec<T, V>::type;
     constexpr uint64_t kChunk = 32ull * V * R;
     const uint32_t lane = threadIdx.x & 31u;
@@ -87,6 +89,9 @@ __global__ void __launch_bounds__(kThreads) k_reshard(const T *__restrict__ src,
             }
         }
     }
+    // launched early behind the previous unit's copy (which touches other
+    // bytes): complete only after it, so that completion stays in order
+    zero_dev::pdl_wait();
 }
 
 }  // namespace
@@ -107,6 +112,10 @@ ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, co
     st = zero_host::sm_count(&sms);
     if (st != ZERO_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    // units after the first launch behind their predecessor (programmatic
+    // dependent launch): they copy disjoint ranges; ZERO_PDL=0 turns it off
+    const char *pdl_env = std::getenv("ZERO_PDL");
+    const bool pdl = !(pdl_env && pdl_env[0] == '0');
     const int vec_bytes = ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15u) == 0;
     for (size_t u = 0; u < to->unit_len.size(); ++u) {
         ReshardArgs r;
@@ -124,16 +133,23 @@ ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, co
         const uint64_t per_thread = (vec ? V : 1) * R;
         const uint64_t blocks = (r.n + per_thread * kThreads - 1) / (per_thread * kThreads);
         const uint32_t grid = uint32_t(std::max<uint64_t>(1, std::min<uint64_t>(blocks, uint64_t(sms) * 8)));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(kThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = (pdl && u > 0) ? 1 : 0;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
         if (elem_bytes == 4) {
             auto *s = static_cast<const uint32_t *>(src);
             auto *d = static_cast<uint32_t *>(dst);
-            if (vec) k_reshard<uint32_t, 4, R><<<grid, kThreads, 0, stream>>>(s, d, r);
-            else k_reshard<uint32_t, 1, R><<<grid, kThreads, 0, stream>>>(s, d, r);
+            cudaLaunchKernelEx(&cfg, vec ? k_reshard<uint32_t, 4, R> : k_reshard<uint32_t, 1, R>, s, d, r);
         } else {
             auto *s = static_cast<const uint16_t *>(src);
             auto *d = static_cast<uint16_t *>(dst);
-            if (vec) k_reshard<uint16_t, 8, R><<<grid, kThreads, 0, stream>>>(s, d, r);
-            else k_reshard<uint16_t, 1, R><<<grid, kThreads, 0, stream>>>(s, d, r);
+            cudaLaunchKernelEx(&cfg, vec ? k_reshard<uint16_t, 8, R> : k_reshard<uint16_t, 1, R>, s, d, r);
         }
         st = zero_host::check_launch("zero_reshard launch");
         if (st != ZERO_OK) return st;
