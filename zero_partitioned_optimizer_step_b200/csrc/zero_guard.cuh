@@ -51,6 +51,7 @@ constexpr int kGuardRB = 8;
 // W32: the fp32 arrays are 32-byte aligned (one 32-byte access per 8 elements).
 template <int VEC, bool OWNER_MAP, bool W32 = false>
 __global__ void __launch_bounds__(kThreads, kGuardMinB) k_reduce(const StepArgs a) {
+    zero_dev::pdl_launch_dependents();
     const uint64_t n = (a.j1 - a.j0) / VEC;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
     double acc = 0.0;
@@ -93,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, kGuardMinB) k_reduce(const StepArgs 
             bad += zero_dev::not_finite(s[e]);
         }
     }
+    zero_dev::pdl_wait();  // predecessor done: its norm slots are final
     zero_dev::block_partials(acc, bad, a);
 }
 
@@ -136,8 +138,14 @@ __global__ void __launch_bounds__(kThreads) k_guard_finalize(const double *ws_no
 
 template <int VEC, bool OWNER_MAP, bool W32 = false>
 __global__ void __launch_bounds__(kThreads, kGuardMinB) k_apply(const StepArgs a, const GuardWord *gw) {
+    // Launched early behind the previous bucket's apply, which itself started
+    // only after the finalize completed, so the guard word is final here.
+    zero_dev::pdl_launch_dependents();
     const GuardWord g = *gw;
-    if (g.skip) return;
+    if (g.skip) {
+        zero_dev::pdl_wait();
+        return;
+    }
     const AdamConsts C = zero_dev::consts_of(a);
     const uint64_t n = (a.j1 - a.j0) / VEC;
     const uint64_t stride = uint64_t(gridDim.x) * kThreads;
@@ -207,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, kGuardMinB) k_apply(const StepArgs a
             for (uint32_t r = 0; r < a.n_prow; ++r) a.params[pi + uint64_t(r) * a.param_stride] = bits;
         }
     }
+    zero_dev::pdl_wait();  // complete only after the predecessor, in stream order
 }
 
 }  // namespace zero_guarded

@@ -683,6 +683,12 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     if (e != cudaSuccess)
         return set_error(ZERO_ECUDA, std::string("zero_step_guarded workspace reset: ") + cudaGetErrorString(e));
     const uint32_t grid = shapes.grid_guard;
+    // Within each pass, launches after the first use programmatic dependent
+    // launch: pass-1 kernels share only the norm slots (added to after the
+    // predecessor completes); a pass-2 kernel starts after its predecessor,
+    // which started after the finalize completed, so the guard word is final.
+    const bool pdl = pdl_enabled();
+    uint32_t n1 = 0, n2 = 0;
     // fp32 arrays 32-byte aligned: 32-byte accesses on the vector path
     const bool w32 = ((reinterpret_cast<uintptr_t>(b->master) | reinterpret_cast<uintptr_t>(b->exp_avg) |
                        reinterpret_cast<uintptr_t>(b->exp_avg_sq) | reinterpret_cast<uintptr_t>(b->reduced_grad)) &
@@ -696,12 +702,11 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             StepArgs y = x;
             y.j0 = j0;
             y.j1 = j1;
-            if (vec && om && w32) zero_guarded::k_reduce<8, true, true><<<grid, kThreads, 0, stream>>>(y);
-            else if (vec && w32) zero_guarded::k_reduce<8, false, true><<<grid, kThreads, 0, stream>>>(y);
-            else if (vec && om) zero_guarded::k_reduce<8, true><<<grid, kThreads, 0, stream>>>(y);
-            else if (vec) zero_guarded::k_reduce<8, false><<<grid, kThreads, 0, stream>>>(y);
-            else if (om) zero_guarded::k_reduce<1, true><<<grid, kThreads, 0, stream>>>(y);
-            else zero_guarded::k_reduce<1, false><<<grid, kThreads, 0, stream>>>(y);
+            const bool dep = pdl && n1++ > 0;
+            auto f = vec ? (w32 ? (om ? zero_guarded::k_reduce<8, true, true> : zero_guarded::k_reduce<8, false, true>)
+                                : (om ? zero_guarded::k_reduce<8, true> : zero_guarded::k_reduce<8, false>))
+                         : (om ? zero_guarded::k_reduce<1, true> : zero_guarded::k_reduce<1, false>);
+            launch_ex(f, grid, kThreads, 0, stream, dep, y);
             return check_launch("zero_step_guarded reduce launch");
         });
         if (st != ZERO_OK) return st;
@@ -733,20 +738,21 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
             StepArgs y = x;
             y.j0 = j0;
             y.j1 = j1;
+            const bool dep = pdl && n2++ > 0;
             if (vec && tma) {
                 const zero_tma::Ring rg = ring_for_launch(ring, j1 - j0, 2, shapes.sms, shapes.tma_smem);
                 const uint64_t tiles = (j1 - j0 + rg.tile - 1) / rg.tile;
                 const uint32_t g = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
                 ApplyKernel f = om ? tma_kernel<true, zero_tma::kReduced>(rg.groups, rg.vw)
                                    : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw);
-                f<<<g, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes, stream>>>(y, rg,
-                                                                                      zero_tma::ApplyExtra{gw});
-            } else if (vec && om && w32) zero_guarded::k_apply<8, true, true><<<grid, kThreads, 0, stream>>>(y, gw);
-            else if (vec && w32) zero_guarded::k_apply<8, false, true><<<grid, kThreads, 0, stream>>>(y, gw);
-            else if (vec && om) zero_guarded::k_apply<8, true><<<grid, kThreads, 0, stream>>>(y, gw);
-            else if (vec) zero_guarded::k_apply<8, false><<<grid, kThreads, 0, stream>>>(y, gw);
-            else if (om) zero_guarded::k_apply<1, true><<<grid, kThreads, 0, stream>>>(y, gw);
-            else zero_guarded::k_apply<1, false><<<grid, kThreads, 0, stream>>>(y, gw);
+                launch_ex(f, g, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes, stream, dep, y, rg,
+                          zero_tma::ApplyExtra{gw});
+            } else {
+                auto f = vec ? (w32 ? (om ? zero_guarded::k_apply<8, true, true> : zero_guarded::k_apply<8, false, true>)
+                                    : (om ? zero_guarded::k_apply<8, true> : zero_guarded::k_apply<8, false>))
+                             : (om ? zero_guarded::k_apply<1, true> : zero_guarded::k_apply<1, false>);
+                launch_ex(f, grid, kThreads, 0, stream, dep, y, static_cast<const zero_guarded::GuardWord *>(gw));
+            }
             return check_launch("zero_step_guarded apply launch");
         });
         if (st != ZERO_OK) return st;

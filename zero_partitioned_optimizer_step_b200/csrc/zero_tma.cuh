@@ -297,7 +297,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float coef = 1.0f;
     if constexpr (SRC == kReduced) {
         const zero_dev::GuardWord g = *x.gw;
-        if (g.skip) return;  // every thread, before any barrier
+        if (g.skip) {  // every thread, before any barrier
+            zero_dev::pdl_wait();
+            return;
+        }
         coef = g.coef;
     }
 
