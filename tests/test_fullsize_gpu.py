@@ -159,13 +159,13 @@ class WindowRun:
         assert self.lp.query(Z.ZERO_Q_LIVE_UNITS) == 0
 
 
-def test_c2_gpt2_small_stage2_ten_steps():
+def test_gpt2_small_stage2_ten_steps():
     r = WindowRun(CONFIGS["gpt2_small"])
     for t in range(1, CONFIGS["gpt2_small"]["steps"] + 1):
         r.step(t, full_norm=(t == 1))
 
 
-def test_c3_stage3_layerwise_five_steps():
+def test_stage3_layerwise_five_steps():
     cfg = CONFIGS["stage3_1p3b"]
     r = WindowRun(cfg)
     n_units = len(cfg["units"])
@@ -175,7 +175,7 @@ def test_c3_stage3_layerwise_five_steps():
     assert r.lp.query(Z.ZERO_Q_PEAK_LIVE_UNITS) == 1
 
 
-def test_c4_single_owner_of_7p5b():
+def test_single_owner_of_7p5b():
     cfg = CONFIGS["owner_7p5b"]
     r = WindowRun(cfg)
     for t in range(1, cfg["steps"] + 1):
@@ -191,7 +191,7 @@ def test_c4_single_owner_of_7p5b():
 
 
 @pytest.mark.parametrize("nd,mb", [(2, 1), (2, 512), (16, 64), (64, 1), (64, 512)])
-def test_c5_bucket_sweep_points(nd, mb):
+def test_bucket_sweep_points(nd, mb):
     cfg = sweep_config(nd, mb)
     r = WindowRun(cfg, seed=nd * 1000 + mb)
     r.step(1)

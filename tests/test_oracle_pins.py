@@ -161,7 +161,7 @@ def test_maps_brute_force_small():
     assert cases > 1000
 
 
-def test_c2_and_c4_plans():
+def test_gpt2_small_and_owner_7p5b_plans():
     # GPT-2-small-shaped flat vector: 12 blocks of (12 h^2 + 13 h), token and
     # position tables, final norm (h = 768, 3072 MLP, 50257 x 768 tokens).
     h = 768

@@ -64,11 +64,11 @@ def test_resume_after_reshard_matches_oracle():
     psi = sum(units)
     c8 = Case(psi, 8, 3, 1 << 16, units=units, config_id=18)
     c8.step_and_compare(1)
-    c4 = Case(psi, 4, 3, 1 << 16, units=units, config_id=18)
-    for src, dst in ((c8.w, c4.w), (c8.m, c4.m), (c8.v, c4.v)):
-        Z.zero_reshard(c8.lp, src, c4.lp, dst)
+    c_to = Case(psi, 4, 3, 1 << 16, units=units, config_id=18)
+    for src, dst in ((c8.w, c_to.w), (c8.m, c_to.m), (c8.v, c_to.v)):
+        Z.zero_reshard(c8.lp, src, c_to.lp, dst)
     Z.zero_stream_status()
-    c4.hw, c4.hm, c4.hv = f32(c4.w), f32(c4.m), f32(c4.v)
+    c_to.hw, c_to.hm, c_to.hv = f32(c_to.w), f32(c_to.m), f32(c_to.v)
     for t in (2, 3):
-        diff = c4.step_and_compare(t)
+        diff = c_to.step_and_compare(t)
         assert all(v == 0 for v in diff.values()), diff
