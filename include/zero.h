@@ -401,9 +401,10 @@ typedef struct zero_peer_bufs {
  * from peers), 12 read + 12 written of local state, 2Nd written to replicas
  * (2(Nd-1) to peers), or 2 at stage 3.  ZERO_EINVAL: as zero_step, or stage
  * 0, Nd > ZERO_MAX_PEERS, rank out of range, a NULL or misaligned entry of
- * grads or params.  ZERO_ECUDA: launch failure.  Aligned bodies run in a
- * 16-byte-load kernel; ZERO_STEP_KERNEL=tma selects the bulk-copy kernel with
- * the rows pulled by 1-D bulk copies from the peers (never multicast). */
+ * grads or params.  ZERO_ECUDA: launch failure.  Aligned bodies run in the
+ * bulk-copy kernel, rows pulled by 1-D bulk copies from the peers (never
+ * multicast), at stage 3, and in a 16-byte-load kernel when replicas are
+ * written; ZERO_STEP_KERNEL=tma|ldg forces either. */
 zero_status_t zero_step_peers(const zero_plan_t *plan, const zero_peer_bufs_t *bufs,
                               const zero_adam_t *adam, uint64_t t, uint64_t first_bucket,
                               uint64_t n_buckets, void *stream);

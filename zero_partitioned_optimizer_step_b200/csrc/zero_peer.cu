@@ -401,17 +401,20 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
             return set_error(ZERO_ECUDA, std::string("zero_step_peers workspace reset: ") + cudaGetErrorString(e));
     }
 
-    // Aligned bodies run in K5 by default; with ZERO_STEP_KERNEL=tma in the
+    // Aligned bodies: where the parameters are written once (stage 3), in the
     // bulk-copy kernel (rows pulled by 1-D bulk copies through the peer table,
-    // no multicast).  With the ranks as allocations on one GPU K5 is faster
-    // (0.85 against 0.82 of copy bandwidth at Nd = 8, 0.74 against 0.61 for
-    // the stage-3 1.3B workload at Nd = 16: a rank's launches are short); the
-    // NVLink rate of either is not measured.  Unaligned edges: K5's scalar twin.
+    // no multicast); with replicas to write, in K5.  Measured with the ranks
+    // as allocations on one GPU, both with programmatic dependent launch: at
+    // stage 3 (1.3B, Nd = 16) 0.945 of copy bandwidth against 0.847 for K5;
+    // with replicas (GPT-2-small, Nd = 8) K5 0.850 against 0.823.  The NVLink
+    // rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg forces
+    // either.  Unaligned edges: K5's scalar twin.
     zero_tma::Ring ring{};
     int *err = nullptr;
     st = zero_detail::wait_error_word(&err);
     if (st != ZERO_OK) return st;
-    const bool tma = zero_ring::kernel_choice() == 2 &&
+    const int choice = zero_ring::kernel_choice();
+    const bool tma = (choice == 2 || (choice == 0 && !replicas)) &&
                      zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring);
     // Vector launches after the first of the call overlap their predecessor
     // (programmatic dependent launch): consecutive launches of one call share
