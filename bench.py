@@ -789,9 +789,14 @@ def run_peer(args, cfg, rank, world, dist):
         return None
     peak, peak_kind = measured_peak()
     hbm_step = Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_STEP)
+    # the library's choice for the aligned bodies (zero_step_peers): the
+    # bulk-copy kernel where parameters are written once, else K5
+    forced = os.environ.get("ZERO_STEP_KERNEL", "")
+    tma = forced == "tma" or (forced != "ldg" and cfg["stage"] == 3)
+    kname = ("k_step_tma through the peer table" if tma else "k_step_peer")
     if world == 1:
         per_launch_bytes = hbm_step / max(1, nd)
-        roof = {"kernel": "k_step_peer (rank r's reduce-scatter + Adam + all-gather over its "
+        roof = {"kernel": kname + " (rank r's reduce-scatter + Adam + all-gather over its "
                           "ranks' buffers; %d calls per step)" % nd,
                 "bound": "hbm", "achieved": hbm_step * args.steps / k_time / 1e9, "peak": peak,
                 "unit": "GB/s", "peak_kind": peak_kind + " (copy bandwidth)", "traffic": None,
@@ -801,7 +806,7 @@ def run_peer(args, cfg, rank, world, dist):
         # per direction: 2(Nd-1)S bytes of peer gradient reads come in and (stages
         # 1-2) as many bytes of replica stores go out; stage-3 stores stay local
         link = 2 * (nd - 1) * S
-        roof = {"kernel": "k_step_peer (one rank per GPU, peer loads and stores over NVLink)",
+        roof = {"kernel": kname + " (one rank per GPU, peer loads and stores over NVLink)",
                 "bound": "nvlink", "achieved": link * args.steps / k_time / 1e9, "peak": NVLINK_GBS,
                 "unit": "GB/s", "peak_kind": "measured peer copy per direction", "traffic": None,
                 "algorithmic_nvlink_bytes_per_direction": link}
