@@ -1,7 +1,10 @@
 // sm_100a kernels of the ZeRO partitioned mixed-precision Adam step, and the
-// C-ABI entry points that launch them.
+// C-ABI entry points that launch them.  K1's default form, the bulk-copy
+// (TMA) ring kernel k_step_tma, is in zero_tma.cuh and its ring shapes in
+// zero_ring.cuh; this file holds K1's 16-byte-load and scalar forms, K2, the
+// launch logic of the step, the guarded step and the layer gathers.
 //
-// K1 k_step_vec8 / k_step_scalar -- one bucket of the step, fused:
+// K1 k_step_tma / k_step_vec8 / k_step_scalar -- one bucket of the step, fused:
 //    reduce-scatter  : g_sum = sum over ranks r = 0..Nd-1 of float(G_r[j]),
 //                      added in rank order from rank 0's value (fp32, RN);
 //    owner Adam      : fp32 master w, first moment m, second moment v;
@@ -18,7 +21,7 @@
 //    master, two moments) and table "三个阶段".
 // K2 k_gather -- stage-3 materialisation of one unit (glossary entry
 //    "临时物化": the shards are briefly put together into the full layer).
-// K3 k_finalize -- sums the per-CTA partials in a fixed order.
+// K3 k_finalize (zero_device.cuh) -- sums the per-CTA partials in a fixed order.
 //
 // Everything is HBM-bound streaming: per element K1 reads 2*Nd bytes of
 // gradients and 12 bytes of state, writes 12 bytes of state and 2*Nd (or 2)
