@@ -54,7 +54,7 @@ def check_against_oracle(psi, nd, stage, bucket, align, units, every_index=True)
     assert t["base"] == op.unit_base and t["off"] == op.unit_offset
     assert t["buckets"] == op.buckets
     idx = range(op.psi_pad) if every_index else \
-        sorted({0, op.psi_pad - 1, *random.Random(psi).sample(range(op.psi_pad), 200)})
+        sorted({0, op.psi_pad - 1, *random.Random(psi).sample(range(op.psi_pad), min(200, op.psi_pad))})
     for p in idx:
         _, o, off, _ = OP.locate(op, p)
         assert lp.query(Z.ZERO_Q_OWNER, p) == o
@@ -254,3 +254,23 @@ def test_plain_c_caller(tmp_path):
         assert got["st3.unit%d" % u] == "%d %d %d" % (o3.unit_pad[u], o3.unit_shard[u], o3.unit_offset[u])
     assert got["st3.release_unheld"] == "%d ESTATE" % Z.ZERO_ESTATE
     assert got["abi"] == "3"
+
+
+try:
+    from hypothesis import HealthCheck, given, settings, strategies as st
+except ImportError:  # pragma: no cover
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=120, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+    @given(nd=st.integers(1, 300), stage=st.integers(0, 3), align=st.sampled_from([1, 2, 3, 8, 64, 100]),
+           units=st.lists(st.integers(1, 5_000_000), min_size=1, max_size=6), data=st.data())
+    def test_plan_matches_oracle_on_random_plans(nd, stage, align, units, data):
+        """Random plans (up to 300 ranks, 6 units, odd alignments and bucket
+        sizes, at most ~2000 buckets each): every table, sampled owners and
+        every byte count as the oracle's maps give them."""
+        psi = sum(units)
+        bucket = data.draw(st.integers(max(1, psi // 2000), max(1, psi + 1000)))
+        check_against_oracle(psi, nd, stage, bucket, align, units if len(units) > 1 else None,
+                             every_index=False)
