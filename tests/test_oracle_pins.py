@@ -536,3 +536,34 @@ def test_reshard_keeps_every_real_element():
         else:
             assert y[o * b.S + off] == 0
     assert np.array_equal(ST.reshard(b, y, a), x)
+
+
+try:
+    from hypothesis import given, settings, strategies as hst
+except ImportError:  # pragma: no cover
+    given = None
+
+if given is not None:
+    @settings(max_examples=60, deadline=None)
+    @given(units=hst.lists(hst.integers(1, 300), min_size=1, max_size=5),
+           a=hst.tuples(hst.integers(1, 12), hst.integers(0, 3), hst.sampled_from([1, 2, 4, 8])),
+           b=hst.tuples(hst.integers(1, 12), hst.integers(0, 3), hst.sampled_from([1, 2, 4, 8])),
+           seed=hst.integers(0, 2 ** 31))
+    def test_reshard_property_random_plans(units, a, b, seed):
+        """For random unit lists and any two plans of them: every real element
+        lands where the destination plan's map puts it, the new padding is
+        zero, and resharding back gives the source bytes."""
+        psi = sum(units)
+        pa = P.make_plan(psi, a[0], a[1], 97, align=a[2], unit_elems=units)
+        pb = P.make_plan(psi, b[0], b[1], 53, align=b[2], unit_elems=units)
+        rng = np.random.default_rng(seed)
+        logical = np.zeros(pa.psi_pad, np.float32)
+        for u, n in enumerate(units):
+            logical[pa.unit_base[u]:pa.unit_base[u] + n] = rng.standard_normal(n)
+        x = ST.logical_to_storage(pa, logical)
+        y = ST.reshard(pa, x, pb)
+        for p in range(pb.psi_pad):
+            u, o, off, j = P.locate(pb, p)
+            want = logical[pa.unit_base[u] + j] if j < units[u] else 0.0
+            assert y[o * pb.S + off] == want
+        assert np.array_equal(ST.reshard(pb, y, pa), x)
