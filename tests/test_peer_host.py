@@ -283,3 +283,14 @@ def test_a_rank_that_leaves_makes_the_next_step_fail_not_hang():
                 p.kill()
     assert res[1] == "left"
     assert res[0].startswith("error:") and res[0].endswith(":no-kernel"), res
+
+
+def test_header_compiles_as_c_and_cpp(tmp_path):
+    """include/zero.h is plain C99 and also valid C++ (extern "C")."""
+    src = tmp_path / "h.c"
+    src.write_text('#include "zero.h"\nint main(void) { return (int)sizeof(zero_peer_bufs_t) == 0; }\n')
+    for cc, std, name in (("gcc", "-std=c99", "h.c"), ("g++", "-std=c++17", "h.cpp")):
+        f = tmp_path / name
+        f.write_text(src.read_text())
+        subprocess.run([cc, std, "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), "-c",
+                        str(f), "-o", str(tmp_path / (name + ".o"))], check=True)
