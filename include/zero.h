@@ -265,10 +265,14 @@ zero_status_t zero_step_buckets(const zero_plan_t *plan,
  * bufs->workspace_bytes are ignored, every other field is as for zero_step.
  * No cudaMalloc, cudaFree or other allocating call is made.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress) and
- * caches it; make that first call before any stream capture.  All calls share
- * the one array: calls whose kernels overlap on the GPU (several streams or
- * threads at once) race on it and must be serialised by the caller.  Each
- * step overwrites the array before reading it, so stale contents are harmless.
+ * caches it; make that first call before any stream capture.  The cached
+ * address belongs to the device's current context: do not reset the device
+ * (cudaDeviceReset) or tear down its primary context between calls, since the
+ * library would keep using the old address.  All calls share the one array:
+ * calls whose kernels overlap on the GPU (several streams or threads at once)
+ * race on it and must be serialised by the caller.  Each step clears the
+ * array on its stream before its kernels add into it, so stale contents are
+ * harmless.
  * ZERO_EINVAL: as zero_step, or a plan whose scratch would exceed the static
  * array (the message says so).  ZERO_ECUDA: the address lookup or a launch
  * failed. */

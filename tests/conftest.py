@@ -6,6 +6,10 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+# The mutation test points this at a copy of the oracle package that holds a
+# planted mistake; the pins then import that copy instead of oracle/.
+if os.environ.get("ORACLE_PKG_ROOT"):
+    sys.path.insert(0, os.environ["ORACLE_PKG_ROOT"])
 
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 

@@ -69,7 +69,6 @@ def test_comm_volume_limits_and_ratio():
             want = rows["stage%d_psi" % st]
             # ring: the printed multiple of Psi times (Nd-1)/Nd, exactly
             assert Fraction(c, psi) == want * Fraction(nd - 1, nd)
-            assert P.comm_bytes_per_rank(pl) == 2 * c
         assert Fraction(per_stage[3], per_stage[0]) == rows["ratio_stage3_over_stage0"]
     # the printed 2 Psi / 3 Psi are the limit as Nd grows
     pl = P.make_plan(psi, 2 ** 20, 3, 2 ** 30, align=1)
@@ -451,9 +450,93 @@ def test_hbm_bytes_per_param():
     pl3 = P.make_plan(sum(units), 16, 3, 1 << 28, unit_elems=units)
     assert pl3.psi_pad == sum(units) and pl3.S == 82_232_704
     assert P.hbm_step_bytes(pl3) == pl3.psi_pad * (2 * 16 + 24 + 2)
-    assert P.hbm_gather_bytes(pl3) == 8 * sum(units)
     pl4 = P.make_plan(7_500_000_000, 64, 2, 25_000_000)
     assert P.hbm_step_bytes(pl4, owner_view=True) == pl4.S * (2 * 64 + 24 + 2)
+
+
+def _ring_reduce_scatter(chunks):
+    """Brute-force ring reduce-scatter.  chunks[r][c]: rank r's piece c (a
+    bf16 tensor).  At step k rank r sends its piece (r-k-1) mod Nd to rank
+    r+1, which adds it to its own; after Nd-1 steps rank r holds the sum of
+    piece r.  Returns (bytes each rank sent, elements each rank sent)."""
+    nd = len(chunks)
+    sent_b, sent_e = [0] * nd, [0] * nd
+    for k in range(nd - 1):
+        msgs = [(r, (r - k - 1) % nd, chunks[r][(r - k - 1) % nd].clone()) for r in range(nd)]
+        for r, c, msg in msgs:
+            sent_b[r] += msg.numel() * msg.element_size()
+            sent_e[r] += msg.numel()
+            chunks[(r + 1) % nd][c] += msg
+    return sent_b, sent_e
+
+
+def _ring_all_gather(chunks):
+    """Brute-force ring all-gather: rank r starts with its piece r valid; at
+    step k it forwards piece (r-k) mod Nd to rank r+1."""
+    nd = len(chunks)
+    sent_b, sent_e = [0] * nd, [0] * nd
+    for k in range(nd - 1):
+        msgs = [(r, (r - k) % nd, chunks[r][(r - k) % nd].clone()) for r in range(nd)]
+        for r, c, msg in msgs:
+            sent_b[r] += msg.numel() * msg.element_size()
+            sent_e[r] += msg.numel()
+            chunks[(r + 1) % nd][c] = msg
+    return sent_b, sent_e
+
+
+@pytest.mark.parametrize("stage", [0, 1, 2, 3])
+@pytest.mark.parametrize("nd,align,units", [(1, 1, [10]), (3, 4, [37, 63, 5]),
+                                            (4, 1, [64]), (5, 2, [3, 1, 40])])
+def test_comm_bytes_equal_bytes_a_brute_force_ring_sends(stage, nd, align, units):
+    """Run the ring collectives of one step on bf16 buffers (per unit: a
+    reduce-scatter of the gradients, then one all-gather of the parameters,
+    or two at stage 3, forward and backward) and count what every rank
+    sends.  The sums and the gathered copies are checked too, with small
+    integers that bf16 holds exactly, so the simulated ring is the real
+    collective."""
+    pl = P.make_plan(sum(units), nd, stage, 1 << 20, align=align, unit_elems=units)
+    sent_b, sent_e = [0] * nd, [0] * nd
+    gen = torch.Generator().manual_seed(nd * 100 + stage)
+    for u, s in enumerate(pl.unit_shard):
+        grads = torch.randint(0, 5, (nd, nd * s), generator=gen).to(torch.bfloat16)
+        chunks = [[grads[r, c * s:(c + 1) * s].clone() for c in range(nd)] for r in range(nd)]
+        b, e = _ring_reduce_scatter(chunks)
+        for r in range(nd):
+            assert torch.equal(chunks[r][r], grads[:, r * s:(r + 1) * s].sum(0))
+            sent_b[r] += b[r]
+            sent_e[r] += e[r]
+        for _ in range(2 if stage == 3 else 1):
+            owned = torch.randint(0, 100, (nd, s), generator=gen).to(torch.bfloat16)
+            chunks = [[owned[c].clone() if c == r else torch.zeros(s, dtype=torch.bfloat16)
+                       for c in range(nd)] for r in range(nd)]
+            b, e = _ring_all_gather(chunks)
+            for r in range(nd):
+                assert all(torch.equal(chunks[r][c], owned[c]) for c in range(nd))
+                sent_b[r] += b[r]
+                sent_e[r] += e[r]
+    assert len(set(sent_b)) == 1 and len(set(sent_e)) == 1
+    assert P.comm_elems_per_rank(pl) == sent_e[0]
+    assert P.comm_bytes_per_rank(pl) == sent_b[0]
+
+
+@pytest.mark.parametrize("nd,align,units", [(3, 4, [37, 63, 5]), (4, 8, [100, 7]),
+                                            (2, 1, [9, 1, 4])])
+def test_gather_bytes_equal_bytes_the_gathers_move(nd, align, units):
+    """Materialise every unit forward, then in reverse, through
+    oracle.step.gather_layer on owner storage filled with distinct ids, and
+    count the bf16 elements each gather reads from the owners' slices (the
+    distinct ids in its output) and writes (its output).  The plans have
+    padding, so counting padded lengths would fail."""
+    pl = P.make_plan(sum(units), nd, 3, 1 << 20, align=align, unit_elems=units)
+    assert pl.psi_pad > sum(units)
+    owner_params = np.arange(nd * pl.S, dtype=np.uint16)
+    moved = 0
+    for u in list(range(len(units))) + list(reversed(range(len(units)))):
+        out = ST.gather_layer(pl, u, owner_params)
+        read = np.unique(out)
+        assert read.size == out.size
+        moved += read.size * owner_params.itemsize + out.nbytes
+    assert P.hbm_gather_bytes(pl) == moved
 
 
 def test_oracle_never_imports_the_product():

@@ -6,7 +6,11 @@ front, or a plain C caller without an allocator: instead of a caller-provided
 workspace, the gradient-norm / overflow scratch is the library's own static
 device array.  This test calls it through the C ABI twice in a row and
 checks every output against zero_step() with a caller-provided workspace on
-the same inputs.  The file is named to run last.
+the same inputs: replicas at stage 2, owner shards of several layers at
+stage 3, and the one-owner view.  Free device memory is read around the
+second call, after the first has loaded the library's static array: an
+allocation of any size inside the call would reserve at least one page of it.
+The file is named to run last.
 """
 import ctypes
 
@@ -19,31 +23,46 @@ from zero_cases import (BF16_ULP, RTOL_NORM, RTOL_REDUCED, RTOL_STATE, Case, bf1
 
 pytestmark = pytest.mark.gpu
 
+CASES = {
+    "stage2_replicas": dict(psi=1_000_003, nd=8, stage=2, bucket=100_000),
+    "stage3_layers": dict(psi=3 * 70_001 + 999, nd=5, stage=3, bucket=50_000,
+                          units=[70_001, 70_001, 70_001, 999]),
+    "owner_view": dict(psi=64 * 20_000, nd=64, stage=2, bucket=300_000, owner_view=5),
+}
 
-def test_noalloc_step_matches_zero_step_on_two_calls():
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_step_matches_zero_step_on_two_calls(name):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
-    ref = Case(1_000_003, 8, 2, 100_000, config_id=2)   # zero_step + workspace
-    new = Case(1_000_003, 8, 2, 100_000, config_id=2)   # zero_step_noalloc
+    kw = dict(CASES[name])
+    args = (kw.pop("psi"), kw.pop("nd"), kw.pop("stage"), kw.pop("bucket"))
+    ref = Case(*args, config_id=2, **kw)   # zero_step + workspace
+    new = Case(*args, config_id=2, **kw)   # zero_step_noalloc
     L = Z.lib()
     for t in (1, 2):
         G = ref.grads(t)
         ref.run_gpu(G, t)
         bufs = Z.make_bufs(new.lp, G, new.w, new.m, new.v, new.params, reduced_grad=new.red,
-                           grad_norm_sq=new.norm, overflow=new.ovf)
+                           grad_norm_sq=new.norm, overflow=new.ovf, owner_view=new.owner)
         adam = Z.make_adam(new.adam)
         stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        torch.cuda.synchronize()
         before = torch.cuda.memory_allocated()
+        free_before = torch.cuda.mem_get_info()[0]
         st = L.zero_step_noalloc(new.lp.handle, ctypes.byref(bufs), ctypes.byref(adam), t, stream)
         assert st == Z.ZERO_OK, L.zero_last_error().decode()
         torch.cuda.synchronize()
         assert torch.cuda.memory_allocated() == before
+        if t == 2:
+            assert torch.cuda.mem_get_info()[0] == free_before
         f32_rel_check(f32(new.w), f32(ref.w), RTOL_STATE, "master")
         f32_rel_check(f32(new.m), f32(ref.m), RTOL_STATE, "exp_avg")
         f32_rel_check(f32(new.v), f32(ref.v), RTOL_STATE, "exp_avg_sq")
         f32_rel_check(f32(new.red), f32(ref.red), RTOL_REDUCED, "reduced")
         bf16_ulp_check(u16(new.params), u16(ref.params), BF16_ULP, "params")
         n_ref, n_new = ref.norm.item(), new.norm.item()
+        assert n_ref > 0
         assert abs(n_new - n_ref) <= RTOL_NORM * n_ref
         assert int(new.ovf.item()) == int(ref.ovf.item()) == 0
 

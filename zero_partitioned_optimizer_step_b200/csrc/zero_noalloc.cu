@@ -71,8 +71,10 @@ ZERO_API zero_status_t zero_step_noalloc(const zero_plan_t *plan, const zero_buf
     void *scratch = nullptr;
     st = scratch_address(&scratch);
     if (st != ZERO_OK) return st;
-    // The step kernels store (not add) every partial on the step's first
-    // launch, so the array's leftover contents need no clearing.
+    // The step kernels add their per-CTA norm partials and non-finite counts
+    // into this array.  zero_step() clears it with cudaMemsetAsync on the
+    // stream before the first bucket's kernel, so whatever an earlier call
+    // left in it does not reach this step's norm or overflow flag.
     zero_bufs_t local = *bufs;
     local.workspace = scratch;
     local.workspace_bytes = kNoAllocScratchBytes;
