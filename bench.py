@@ -1,7 +1,7 @@
 """Benchmark of the ZeRO partitioned optimizer step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config gpt2_small|toy|stage3_1p3b|owner_7p5b|sweep]
+                    [--config sweep|gpt2_small|toy|stage3_1p3b|owner_7p5b]
                     [--nd ND --bucket-mb MB]                 # one bucket-sweep point
                     [--sweep OUT.jsonl]                      # the whole bucket sweep
                     [--eager]                                # launch every step from the host
@@ -12,11 +12,14 @@ gradient-norm / overflow reduction (stage 3 workloads add the forward and
 backward layer gathers).  The timed steps are replayed as a CUDA graph
 (graph.StepGraph: the same kernels, with the step's constants refreshed in
 device memory by a captured copy) unless the workload gathers layers or
---eager is given; the dominant kernel's own rate is then taken from extra
-eager steps with an event around every bucket.  The default workload is the
-GPT-2-small-shaped flat vector (124,439,808 parameters, Nd = 8 logical
-ranks, stage 2, 25M-element buckets).  Inputs are resident in HBM when timing starts and one
-step touches ~7 GB, far more than the 126 MB L2, so no flush is needed.
+--eager is given.  The dominant kernel's rate is timed in the same steps: an
+event pair around each step's chain of bucket kernels (which start one
+another early through programmatic dependent launch) gives the chain's span,
+divided by its launches.  The default workload is one point of the
+bucket-size sweep: 5e8 parameters, Nd = 16 logical ranks, stage 2, buckets
+of 64 MB of one rank's bf16 gradient (2^25 elements; 15 buckets).  Inputs
+are resident in HBM when timing starts and one step touches ~44 GB, far more
+than the 126 MB L2, so no flush is needed.
 
 The metric is parameters updated per second (Gparams/s); the JSON line also
 carries the achieved HBM bandwidth of the dominant kernel against the measured
@@ -44,7 +47,8 @@ if ROOT not in sys.path:
 METRIC = "Gparams/s per ZeRO step (RS+Adam+AG); achieved HBM GB/s vs B200 peak"
 UNIT = "Gparams/s"
 FALLBACK_HBM_GBS = 6650.0
-K1_PROFILE = os.path.join(ROOT, "profiles", "k_step_tma_gpt2_small_nd8.md")
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e, nominal
+PROFILES = os.path.join(ROOT, "profiles")
 K1_SOURCES = [os.path.join(ROOT, "zero_partitioned_optimizer_step_b200", "csrc", f)
               for f in ("zero_step.cu", "zero_tma.cuh", "zero_ring.cuh", "zero_device.cuh")]
 
@@ -64,10 +68,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="gpt2_small",
-                    choices=["toy", "gpt2_small", "stage3_1p3b", "owner_7p5b", "sweep"])
+    ap.add_argument("--config", default="sweep",
+                    choices=["sweep", "toy", "gpt2_small", "stage3_1p3b", "owner_7p5b"])
     ap.add_argument("--nd", type=int, default=None,
-                    help="logical ranks (bucket sweep point: default 64; other workloads: "
+                    help="logical ranks (bucket sweep point: default 16; other workloads: "
                          "override their Nd)")
     ap.add_argument("--bucket-mb", type=int, default=64)
     ap.add_argument("--sweep", default=None, help="write the bucket sweep grid as JSON lines here")
@@ -107,7 +111,7 @@ def parse_args():
 def get_cfg(args):
     from zero_partitioned_optimizer_step_b200.configs import CONFIGS, sweep_config
     if args.config == "sweep":
-        cfg = sweep_config(args.nd or 64, args.bucket_mb)
+        cfg = sweep_config(args.nd or 16, args.bucket_mb)
     else:
         cfg = dict(CONFIGS[args.config])
         if args.nd is not None:
@@ -146,18 +150,28 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def k1_traffic_per_elem():
-    """dram bytes per element of the vector kernel from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
+def k1_traffic_per_elem(kernel, nd, bucket_elems, view):
+    """DRAM bytes per element of one bucket launch, from a committed ncu
+    summary of the same kernel on a launch of the same shape (kernel, Nd,
+    bucket size, view), if it was taken on the current kernel source (else
+    None).  A summary states its shape as `shape: <kernel> nd=<Nd>
+    bucket_elems=<n> view=<replicas|owner>`."""
+    want = "%s nd=%d bucket_elems=%d view=%s" % (kernel, nd, bucket_elems, view)
+    src_hash = kernel_source_hash()
     try:
-        txt = open(K1_PROFILE, encoding="utf-8").read()
-        src_hash = kernel_source_hash()
+        names = sorted(os.listdir(PROFILES))
+    except OSError:
+        return None
+    for name in names:
+        if not name.endswith(".md"):
+            continue
+        with open(os.path.join(PROFILES, name), encoding="utf-8") as f:
+            txt = f.read()
+        sh = re.search(r"^shape:\s*(.+?)\s*$", txt, re.M)
         m = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
         b = re.search(r"dram_bytes_per_element:\s*([0-9.eE+-]+)", txt)
-        if m and b and m.group(1) == src_hash:
+        if sh and m and b and sh.group(1) == want and m.group(1) == src_hash:
             return float(b.group(1))
-    except OSError:
-        pass
     return None
 
 
@@ -328,14 +342,20 @@ class Workload:
         a = U + self.owner * s
         return max(0, min(hi, a + s) - max(lo, a))
 
-    def step(self, t, stream, events=None):
+    def step(self, t, stream, events=None, span=None):
         """One step; with `events` (list of nb+1 CUDA events) each bucket's
-        launch is bracketed so the vector kernel can be timed per launch."""
+        launch is bracketed so the vector kernel can be timed per launch; with
+        `span` (two events) the step's bucket chain is bracketed as a whole
+        (the layer gathers of stage 3 come after the second event)."""
         Z = self.Z
         kw = dict(grad_norm_sq=self.norm, overflow=self.ovf, workspace=self.ws,
                   owner_view=self.owner, stream=stream)
         if events is None:
+            if span is not None:
+                span[0].record(stream)
             Z.zero_step(self.lp, self.G, self.w, self.m, self.v, self.params, self.adam, t, **kw)
+            if span is not None:
+                span[1].record(stream)
         else:
             for i, (lo, hi, _) in enumerate(self.chunks):
                 events[i].record(stream)
@@ -411,6 +431,42 @@ def cpu_baseline(wl, budget_s=10.0):
                       % (wins, win, wl.cfg["nd"], done, t_compute)}
 
 
+def cpu_baseline_threads(wl, budget_s=5.0):
+    """The same oracle core, unchanged, on every host core this process may
+    use: each round copies one 2^22-column window of the step to the host,
+    cuts it into one contiguous column block per core, and runs the oracle's
+    update on all blocks at once from a thread pool (the C core runs without
+    the interpreter lock).  Columns are independent, so the blocks need no
+    coordination.  Timed: the concurrent section of each round, until
+    ~budget_s of wall time."""
+    import numpy as np
+    import torch
+    from concurrent.futures import ThreadPoolExecutor
+    from oracle import core
+    cores = len(os.sched_getaffinity(0))
+    win = min(1 << 22, wl.elems)
+    n_win = max(1, wl.elems // win)
+    done, rounds, t_wall = 0, 0, 0.0
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        while t_wall < budget_s:
+            lo = (rounds % n_win) * win
+            G = wl.G[:, lo:lo + win].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+            state = [x[lo:lo + win].cpu().numpy() for x in (wl.w, wl.m, wl.v)]
+            cuts = np.linspace(0, win, cores + 1).astype(np.int64)
+            blocks = [(np.ascontiguousarray(G[:, a:b]), *[x[a:b].copy() for x in state])
+                      for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+            t1 = time.perf_counter()
+            list(ex.map(lambda blk: core.update(blk[0], blk[1], blk[2], blk[3], wl.adam, 1), blocks))
+            t_wall += time.perf_counter() - t1
+            done += win
+            rounds += 1
+    return {"value": done / t_wall / 1e9, "unit": UNIT, "cores": cores,
+            "kind": "oracle, all cores (threads over disjoint column blocks)",
+            "sample": "%d windows of %d columns x %d gradient rows (%d params, %.1f s of wall time "
+                      "on %d threads; host copies not timed)"
+                      % (rounds, win, wl.cfg["nd"], done, t_wall, cores)}
+
+
 def run_reference(args, cfg):
     """Reference arm: the CPU oracle timed on the host cores, K steps of a
     bounded sample (2^22 columns of the workload, all Nd gradient rows)."""
@@ -468,9 +524,9 @@ def run_ours(args, cfg, rank, world, dist):
             t += 1
     torch.cuda.synchronize()
 
-    n_ev = args.steps if sg is None else min(args.steps, 50)
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.chunks) + 1)]
-              for _ in range(n_ev)]
+    # one event pair per timed step around its chain of bucket kernels
+    spans = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index).start()
@@ -482,37 +538,46 @@ def run_ours(args, cfg, rank, world, dist):
     t0 = t
     for k in range(args.steps):
         if sg is not None:
+            spans[k][0].record(stream)
             sg.replay(t0 + k)
+            spans[k][1].record(stream)
         else:
-            wl.step(t0 + k, stream, events[k])
+            wl.step(t0 + k, stream, span=spans[k])
     end.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
     elapsed = start.elapsed_time(end) / 1e3
-    if sg is not None:
-        # the kernel's own rate, from eager steps with an event per bucket
-        for k in range(n_ev):
-            wl.step(t0 + args.steps + k, stream, events[k])
-        torch.cuda.synchronize()
-    # dominant kernel: the fused bucket kernel, timed per launch
-    k1_time = 0.0
-    k1_elems = 0
-    for k in range(n_ev):
-        for i, (_, _, n) in enumerate(wl.chunks):
-            k1_time += events[k][i].elapsed_time(events[k][i + 1]) / 1e3
-            k1_elems += n
+    # dominant kernel: the fused bucket kernel, in the timed steps themselves
+    k1_time = sum(a.elapsed_time(b) for a, b in spans) / 1e3
+    k1_elems = args.steps * sum(n for _, _, n in wl.chunks)
+    # for context: the same kernel launched alone (an event around every
+    # bucket, which also stops each launch from starting during the last)
+    n_iso = min(args.steps, 20)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.chunks) + 1)]
+              for _ in range(n_iso)]
+    for k in range(n_iso):
+        wl.step(t0 + args.steps + k, stream, events[k])
+    torch.cuda.synchronize()
+    iso_time = sum(events[k][i].elapsed_time(events[k][i + 1]) / 1e3
+                   for k in range(n_iso) for i in range(len(wl.chunks)))
+    iso = (iso_time, n_iso * sum(n for _, _, n in wl.chunks), n_iso * len(wl.chunks))
     elapsed = max_over_ranks(elapsed, dist, dev)
 
     # end to end through the public API: gradients from pinned host memory
     # every step, the step, the norm and overflow flag read back every step
     e2e = None
     if not args.no_e2e:
-        e2e = _e2e(args, wl, stream, dev, world, dist, t0 + args.steps + n_ev)
+        e2e = _e2e(args, wl, stream, dev, world, dist, t0 + args.steps + n_iso)
     if rank != 0:
         return None
-    res = _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=n_ev)
+    timing = ("graph-replayed" if sg is not None else "host-launched") + \
+        " timed steps: an event pair around each step's chain of bucket kernels (with the " \
+        "workspace reset and the one-CTA finalize, and in a graph the constants copy), " \
+        "divided by the chain's launches"
+    res = _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, timing=timing,
+                  isolated=iso)
     res["config"]["graph"] = sg is not None
     res["config"]["weight_decay"] = args.weight_decay
     if wl.layer is not None:
@@ -630,7 +695,8 @@ def run_guarded(args, cfg, rank, world, dist):
 def _e2e(args, wl, stream, dev, world, dist, t_first):
     import torch
     e2e_steps = max(1, min(args.e2e_steps, args.steps))
-    Gh = wl.G.cpu().pin_memory()
+    Gh = torch.empty(wl.G.shape, dtype=wl.G.dtype, pin_memory=True)
+    Gh.copy_(wl.G)
     out_h = torch.empty(2, dtype=torch.float64).pin_memory()
     ovf_h = torch.empty(1, dtype=torch.int32).pin_memory()
     e0 = torch.cuda.Event(enable_timing=True)
@@ -653,21 +719,32 @@ def _e2e(args, wl, stream, dev, world, dist, t_first):
             "d2h_bytes_per_step": 8 + 4, "steps": e2e_steps}
 
 
-def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=None):
+def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, timing, isolated=None):
+    """The JSON line.  k1_time / k1_elems: the bucket kernels' time and
+    elements over the timed steps (`timing` says how they were timed);
+    isolated: (time, elements, launches) of the same kernel timed launch by
+    launch, for context, or None."""
     peak, peak_kind = measured_peak()
     per_elem = wl.step_bytes / wl.elems
     k1_bytes = per_elem * k1_elems
     achieved = k1_bytes / k1_time / 1e9
-    n_launch = (n_ev or args.steps) * len(wl.chunks)
-    tr = (k1_traffic_per_elem() if (args.config == "gpt2_small" and args.psi is None
-                                    and wl.Z.zero_step_kernel(wl.lp, wl.owner) == "k_step_tma") else None)
+    n_launch = args.steps * len(wl.chunks)
     kname = wl.Z.zero_step_kernel(wl.lp, wl.owner)
+    view = "owner" if wl.owner >= 0 else "replicas" if wl.replicas else "shards"
+    tr = k1_traffic_per_elem(kname, cfg["nd"], cfg["bucket_elems"], view)
     roof = {"kernel": kname + " (fused reduce-scatter + Adam + all-gather, one bucket)",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
+            "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
             "traffic": None if tr is None else tr * k1_elems / n_launch,
             "algorithmic_bytes_per_launch": k1_bytes / n_launch,
-            "avg_launch_ms": k1_time / n_launch * 1e3}
+            "avg_launch_ms": k1_time / n_launch * 1e3, "timing": timing}
+    if isolated is not None:
+        it, ie, il = isolated
+        a_iso = per_elem * ie / it / 1e9
+        roof["isolated"] = {"avg_launch_ms": it / il * 1e3, "achieved": a_iso, "frac": a_iso / peak,
+                            "timing": "host-launched steps with an event around every bucket "
+                                      "(no launch starts while the previous one drains)"}
     step_bytes = wl.step_bytes + wl.gather_bytes
     value = job_value(world, wl.params_per_step, args.steps, elapsed)
     out = {
@@ -676,6 +753,7 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=Non
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": cfg["workload"], "psi": cfg["psi"], "nd": cfg["nd"],
+                   "precision": "bf16 gradients and parameters; fp32 master, m, v and arithmetic",
                    "stage": cfg["stage"], "bucket_elems": cfg["bucket_elems"],
                    "owner_view": cfg["owner_view"], "buckets": wl.nb,
                    "hbm_bytes_per_step": step_bytes,
@@ -689,6 +767,7 @@ def _report(args, cfg, wl, world, elapsed, k1_time, k1_elems, clk, e2e, n_ev=Non
     }
     if not args.no_cpu_baseline and world == 1:
         out["cpu_baseline"] = cpu_baseline(wl)
+        out["cpu_baseline_all_cores"] = cpu_baseline_threads(wl)
     return out
 
 
@@ -932,26 +1011,33 @@ def run_sweep(args, rank, world, dist):
                     wl.step(t, stream)
                 s0 = torch.cuda.Event(enable_timing=True)
                 s1 = torch.cuda.Event(enable_timing=True)
+                spans = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                         for _ in range(args.steps)]
                 torch.cuda.synchronize()
                 s0.record(stream)
                 for k in range(args.steps):          # the step as a user runs it
-                    wl.step(args.warmup + 1 + k, stream)
+                    wl.step(args.warmup + 1 + k, stream, span=spans[k])
                 s1.record(stream)
                 torch.cuda.synchronize()
                 elapsed = s0.elapsed_time(s1) / 1e3
-                # again with an event around every bucket, for the kernel's own rate
+                k1_time = sum(a.elapsed_time(b) for a, b in spans) / 1e3
+                k1_elems = args.steps * sum(n for _, _, n in wl.chunks)
+                # again with an event around every bucket: each launch alone
                 events = [[torch.cuda.Event(enable_timing=True) for _ in range(len(wl.chunks) + 1)]
                           for _ in range(args.steps)]
                 for k in range(args.steps):
                     wl.step(args.warmup + args.steps + 1 + k, stream, events[k])
                 torch.cuda.synchronize()
-                k1_time = sum(events[k][i].elapsed_time(events[k][i + 1]) / 1e3
-                              for k in range(args.steps) for i in range(len(wl.chunks)))
-                k1_elems = args.steps * sum(n for _, _, n in wl.chunks)
+                iso_time = sum(events[k][i].elapsed_time(events[k][i + 1]) / 1e3
+                               for k in range(args.steps) for i in range(len(wl.chunks)))
+                iso = (iso_time, k1_elems, args.steps * len(wl.chunks))
                 a = argparse.Namespace(**vars(args))
                 a.config = "sweep"
                 a.no_cpu_baseline = True
-                res = _report(a, cfg, wl, world, elapsed, k1_time, k1_elems, None, None)
+                timing = ("host-launched steps: an event pair around each step's chain of bucket "
+                          "kernels, divided by the chain's launches")
+                res = _report(a, cfg, wl, world, elapsed, k1_time, k1_elems, None, None,
+                              timing=timing, isolated=iso)
                 res["config"]["bucket_mb"] = mb
                 if args.graph:
                     sg = wl.make_graph()
@@ -976,6 +1062,7 @@ def run_sweep(args, rank, world, dist):
                 print(json.dumps({"nd": nd, "mb": mb, "value": res["value"],
                                   "step_gbs": res["hbm_gbs"], "k1_gbs": res["roofline"]["achieved"],
                                   "k1_frac": res["roofline"]["frac"],
+                                  "k1_isolated_frac": res["roofline"]["isolated"]["frac"],
                                   "graph_value": (res.get("graph") or {}).get("value")}), flush=True)
             del wl
             torch.cuda.empty_cache()

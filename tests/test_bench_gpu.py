@@ -48,10 +48,17 @@ def test_bench_line(mode):
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
     assert line["gpu_launches"] > 0
     assert line["clocks"] is None or "sm_mhz" in line["clocks"]
+    if mode in ("default", "eager"):
+        # the kernel is timed in the timed steps: its launches fit in the step
+        assert roof["avg_launch_ms"] * line["config"]["buckets"] <= line["ms_per_step"] * 1.001
+        assert "timing" in roof and roof["isolated"]["frac"] > 0
+        assert abs(roof["frac_of_nominal"] * roof["nominal_peak"] - roof["achieved"]) < 1e-6
     if mode == "default":
         assert line["config"]["graph"] is True
         assert line["e2e"]["h2d_bytes_per_step"] > 0 and line["e2e"]["value"] > 0
         assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] > 0
+        allc = line["cpu_baseline_all_cores"]
+        assert allc["cores"] >= 1 and allc["value"] > 0
     if mode == "eager":
         assert line["config"]["graph"] is False
     if mode == "stage3_prefetch":

@@ -16,7 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libzero.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("zero_plan.cpp", "zero_step.cu", "zero_noalloc.cu", "zero_peer.cu", "zero_reshard.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("zero_internal.h", "zero_device.cuh", "zero_tma.cuh",
-                                             "zero_guard.cuh", "zero_host.cuh", "zero_ring.cuh")] + \
+                                             "zero_guard.cuh", "zero_host.cuh", "zero_ring.cuh",
+                                             "zero_trace.h")] + \
     [os.path.join(ROOT, "include", "zero.h")]
 
 NVCC_FLAGS = [

@@ -50,6 +50,7 @@
 #include "zero_internal.h"
 #include "zero_ring.cuh"
 #include "zero_tma.cuh"
+#include "zero_trace.h"
 
 using zero_detail::set_error;
 using zero_host::aligned16;
@@ -354,6 +355,8 @@ zero_status_t validate_peers(const zero_plan_t *p, const zero_peer_bufs_t *b, co
 ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_bufs_t *b, const zero_adam_t *adam,
                                        uint64_t t, uint64_t first, uint64_t count, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_step_peers t=%llu buckets [%llu, %llu)", (unsigned long long)t,
+                                 (unsigned long long)first, (unsigned long long)(first + count));
     zero_status_t st = validate_peers(p, b, adam, t);
     if (st != ZERO_OK) return st;
     if (first > p->n_buckets || count > p->n_buckets - first)
@@ -470,6 +473,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         a.q_shift = replicas ? 0 : a.s_shift;
         const bool vec_ok = mult8(a.s_shift);
         const uint64_t vlo = (p0 + 7) & ~uint64_t(7), vhi = p1 & ~uint64_t(7);
+        const zero_trace::Range rb("bucket %llu", (unsigned long long)bk);
         if (!vec_ok || vlo >= vhi) {
             st = launch(p0, p1, false);
         } else {
@@ -480,6 +484,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         if (st != ZERO_OK) return st;
     }
     if (want_ws && first + count == p->n_buckets && count > 0) {
+        const zero_trace::Range rf("norm finalize");
         k_finalize<<<1, kThreads, 0, stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots, b->grad_norm_sq,
                                                b->overflow);
         st = check_launch("zero_step_peers finalize launch");
@@ -491,6 +496,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
 ZERO_API zero_status_t zero_gather_layer_peers(zero_plan_t *p, uint32_t unit, const void *const *owner_params,
                                                void *full_layer, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_gather_layer_peers unit %u", unit);
     if (!p) return set_error(ZERO_EINVAL, "zero_gather_layer_peers: NULL plan");
     if (p->stage != 3) return set_error(ZERO_EINVAL, "zero_gather_layer_peers: only stage 3 materialises layers");
     if (p->nd > ZERO_MAX_PEERS) return set_error(ZERO_EINVAL, "zero_gather_layer_peers: nd exceeds ZERO_MAX_PEERS");

@@ -14,6 +14,7 @@
 #include <new>
 
 #include "zero_internal.h"
+#include "zero_trace.h"
 
 using zero_detail::set_error;
 
@@ -305,6 +306,7 @@ ZERO_API zero_status_t zero_release_layer(zero_plan_t *p, uint32_t unit) {
     p->live[unit] = 0;
     p->n_live -= 1;
     p->live_bytes -= 2 * p->unit_len[unit];
+    zero_trace::mark("zero_release_layer unit %u", unit);
     return ZERO_OK;
 }
 

@@ -12,6 +12,7 @@
 #include "zero_device.cuh"
 #include "zero_host.cuh"
 #include "zero_internal.h"
+#include "zero_trace.h"
 
 using zero_detail::set_error;
 
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kThreads) k_reshard(const T *__restrict__ src,
 ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, const zero_plan_t *to, void *dst,
                                     uint32_t elem_bytes, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_reshard %u-byte elements", elem_bytes);
     if (!from || !to || !src || !dst) return set_error(ZERO_EINVAL, "zero_reshard: NULL argument");
     if (elem_bytes != 2 && elem_bytes != 4)
         return set_error(ZERO_EINVAL, "zero_reshard: elem_bytes must be 2 (bf16) or 4 (fp32)");
@@ -127,6 +129,7 @@ ZERO_API zero_status_t zero_reshard(const zero_plan_t *from, const void *src, co
         r.jump_b = to->S - r.s_b;
         r.n = uint64_t(to->nd) * r.s_b;
         r.len = to->unit_len[u];
+        const zero_trace::Range ru("reshard unit %zu", u);
         const uint64_t V = 16 / elem_bytes;
         const bool vec = vec_bytes && ((r.off_a | r.s_a | r.jump_a | r.off_b | r.s_b | r.jump_b) % V) == 0;
         constexpr int R = 8;

@@ -51,6 +51,7 @@
 #include "zero_ring.cuh"
 #include "zero_host.cuh"
 #include "zero_internal.h"
+#include "zero_trace.h"
 
 using zero_detail::set_error;
 using zero_host::aligned16;
@@ -529,6 +530,8 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
                                          const zero_adam_t *adam, uint64_t t, uint64_t first,
                                          uint64_t count, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_step t=%llu buckets [%llu, %llu)", (unsigned long long)t,
+                                 (unsigned long long)first, (unsigned long long)(first + count));
     zero_status_t st = validate_step(p, b, adam, t);
     if (st != ZERO_OK) return st;
     if (first > p->n_buckets || count > p->n_buckets - first)
@@ -561,10 +564,12 @@ ZERO_API zero_status_t zero_step_buckets(const zero_plan_t *p, const zero_bufs_t
         StepArgs x;
         bool owner_map, vec_ok;
         if (!bucket_args(p, b, a, bk, &x, &owner_map, &vec_ok)) continue;
+        const zero_trace::Range r("bucket %llu", (unsigned long long)bk);
         st = L.run(x, owner_map, vec_ok);
         if (st != ZERO_OK) return st;
     }
     if (L.want_ws && first + count == p->n_buckets && count > 0) {
+        const zero_trace::Range r("norm finalize");
         k_finalize<<<1, kThreads, 0, L.stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots, b->grad_norm_sq,
                                                  b->overflow);
         st = check_launch("zero_step finalize launch");
@@ -585,6 +590,7 @@ ZERO_API zero_status_t zero_step(const zero_plan_t *p, const zero_bufs_t *b, con
 ZERO_API zero_status_t zero_gather_layer(zero_plan_t *p, uint32_t unit, const void *owner_params,
                                          void *full_layer, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_gather_layer unit %u", unit);
     if (!p) return set_error(ZERO_EINVAL, "zero_gather_layer: NULL plan");
     if (p->stage != 3) return set_error(ZERO_EINVAL, "zero_gather_layer: only stage 3 materialises layers");
     if (unit >= p->unit_len.size()) return set_error(ZERO_EINVAL, "zero_gather_layer: unit out of range");
@@ -662,6 +668,7 @@ ZERO_API zero_status_t zero_step_kernel(const zero_plan_t *p, int32_t owner_view
 ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t *b, const zero_adam_t *adam,
                                          const zero_guard_t *guard, uint64_t t, void *stream_) {
     zero_detail::clear_error();
+    const zero_trace::Range call("zero_step_guarded t=%llu", (unsigned long long)t);
     zero_status_t st = validate_step(p, b, adam, t);
     if (st != ZERO_OK) return st;
     if (!guard) return set_error(ZERO_EINVAL, "zero_step_guarded: NULL guard");
@@ -701,6 +708,7 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
         StepArgs x;
         bool om, vec_ok;
         if (!bucket_args(p, b, a, bk, &x, &om, &vec_ok)) continue;
+        const zero_trace::Range r("reduce bucket %llu", (unsigned long long)bk);
         st = split_launch(x, vec_ok, [&](uint64_t j0, uint64_t j1, bool vec) -> zero_status_t {
             StepArgs y = x;
             y.j0 = j0;
@@ -714,12 +722,15 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
         });
         if (st != ZERO_OK) return st;
     }
-    zero_guarded::k_guard_finalize<<<1, kThreads, 0, stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots,
-                                                             b->grad_norm_sq, b->overflow, gw,
-                                                             guard->max_grad_norm, adam->grad_scale,
-                                                             guard->skip_nonfinite ? 1 : 0);
-    st = check_launch("zero_step_guarded finalize launch");
-    if (st != ZERO_OK) return st;
+    {
+        const zero_trace::Range fin("guard finalize");
+        zero_guarded::k_guard_finalize<<<1, kThreads, 0, stream>>>(a.ws_norm, a.ws_bad, zero_detail::kMaxSlots,
+                                                                 b->grad_norm_sq, b->overflow, gw,
+                                                                 guard->max_grad_norm, adam->grad_scale,
+                                                                 guard->skip_nonfinite ? 1 : 0);
+        st = check_launch("zero_step_guarded finalize launch");
+        if (st != ZERO_OK) return st;
+    }
     // pass 2: Adam from the reduced gradients (no-op when the step is skipped).
     // When the parameters are written once (stage 3), aligned bodies run in
     // the bulk-copy kernel with the reduced gradient as its one fp32 row (a
@@ -737,6 +748,7 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
         StepArgs x;
         bool om, vec_ok;
         if (!bucket_args(p, b, a, bk, &x, &om, &vec_ok)) continue;
+        const zero_trace::Range r("apply bucket %llu", (unsigned long long)bk);
         st = split_launch(x, vec_ok, [&](uint64_t j0, uint64_t j1, bool vec) -> zero_status_t {
             StepArgs y = x;
             y.j0 = j0;
