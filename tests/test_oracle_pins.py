@@ -200,6 +200,38 @@ def test_bf16_rne_matches_torch():
     assert np.array_equal(core.bf16_rne(back), ours[~nan])
 
 
+def test_bf16_rne_matches_torch_on_every_pattern():
+    """All 2^32 fp32 bit patterns, in chunks of 2^24: the same bf16 as
+    torch's conversion for every non-NaN input; every NaN stays a quiet NaN
+    with its sign."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    chunk = 1 << 22
+
+    def check(c):
+        bits = np.arange(c * chunk, (c + 1) * chunk, dtype=np.uint64).astype(np.uint32)
+        x = bits.view(np.float32)
+        ours = core.bf16_rne(x)
+        theirs = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        nan = np.isnan(x)
+        if nan.any():
+            q = ours[nan]
+            if not (np.all((q & 0x7F80) == 0x7F80) and np.all((q & 0x0040) != 0)
+                    and np.array_equal(q >> 15, (bits[nan] >> 31).astype(np.uint16))):
+                return c
+            ours, theirs = ours[~nan], theirs[~nan]
+        return None if np.array_equal(ours, theirs) else c
+
+    threads = torch.get_num_threads()
+    torch.set_num_threads(1)          # the chunks run side by side instead
+    try:
+        with ThreadPoolExecutor(max_workers=max(1, len(os.sched_getaffinity(0)))) as ex:
+            bad = [c for c in ex.map(check, range(1 << 10)) if c is not None]
+    finally:
+        torch.set_num_threads(threads)
+    assert not bad, bad
+
+
 # ------------------------------------------------------------ reduction
 def test_reduce_rank_order_cancellation():
     two25 = np.float32(2.0 ** 25)
