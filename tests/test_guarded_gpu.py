@@ -51,11 +51,14 @@ def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align, kern
         assert torch.equal(a.params.view(torch.int16), b.params.view(torch.int16))
 
 
-@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+@pytest.mark.parametrize("kernel", ["tma", "ldg", "tma16"])
 @pytest.mark.parametrize("psi,nd,stage,units", [(500_000, 8, 2, None),
                                                 (300_001, 16, 3, [100_000, 3, 199_998])])
 def test_guarded_clipping(psi, nd, stage, units, kernel, monkeypatch):
-    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
+    """tma16: the second pass in the bulk-copy kernel with 16 consumer warps."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel[:3])
+    if kernel == "tma16":
+        monkeypatch.setenv("ZERO_TMA_CW", "16")
     c = Case(psi, nd, stage, 1 << 15, units=units, sigma=1e-2, config_id=14, adam=ADAMW)
     for t in (1, 2, 3):
         diff, coef, skipped = c.guarded_step_and_compare(t, 0.05, True)

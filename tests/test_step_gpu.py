@@ -235,14 +235,17 @@ def test_kernels_agree_bitwise_large_nd():
         assert outs[0][5] == pytest.approx(outs[1][5], rel=1e-12)
 
 
+@pytest.mark.parametrize("cw", ["8", "16"])
 @pytest.mark.parametrize("vw", ["2", "4", "8"])
 @pytest.mark.parametrize("psi,nd,stage,units,owner", [
     (700_001, 8, 2, None, -1), (600_000, 16, 3, [200_000, 1_000, 399_000], -1),
-    (500_000, 64, 2, None, 7)])
-def test_bulk_kernel_vector_widths(vw, psi, nd, stage, units, owner, monkeypatch):
-    """The bulk-copy kernel with 2, 4 and 8 elements per consumer thread."""
+    (500_000, 64, 2, None, 7), (300_007, 2, 2, None, -1)])
+def test_bulk_kernel_vector_widths(cw, vw, psi, nd, stage, units, owner, monkeypatch):
+    """The bulk-copy kernel with 2, 4 and 8 elements per consumer thread, and
+    8 or 16 consumer warps."""
     monkeypatch.setenv("ZERO_STEP_KERNEL", "tma")
     monkeypatch.setenv("ZERO_TMA_VW", vw)
+    monkeypatch.setenv("ZERO_TMA_CW", cw)
     c = Case(psi, nd, stage, 1 << 18, units=units, owner_view=owner, config_id=11)
     for t in (1, 2):
         diff = c.step_and_compare(t)

@@ -418,7 +418,8 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
     if (st != ZERO_OK) return st;
     const int choice = zero_ring::kernel_choice();
     const bool tma = (choice == 2 || (choice == 0 && !replicas)) &&
-                     zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring);
+                     zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring,
+                                            zero_tma::kConsumerWarps);
     // Vector launches after the first of the call overlap their predecessor
     // (programmatic dependent launch): consecutive launches of one call share
     // only the norm slots, which every kernel adds to after its predecessor

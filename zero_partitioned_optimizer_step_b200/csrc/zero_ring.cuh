@@ -30,11 +30,14 @@ inline uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127
 // at which an SM completes such copies caps the read bandwidth (0.64 of copy
 // bandwidth against 0.80 for the load kernel, one owner of 64 ranks).  With
 // two groups the stage count is even (each group owns half the stages).
-// ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS / ZERO_TMA_VW override the
+// ZERO_TMA_CW=16 runs 16 consumer warps instead of 8 (where the caller has
+// such kernels; the per-thread vector width shrinks so every thread keeps
+// work).  ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS / ZERO_TMA_VW override the
 // shape (tuning; a tile must be a positive multiple of 256).  `err` is the
 // device error word the kernel's bounded waits report to.
 inline zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t groups) {
     zero_tma::Ring q{};
+    q.cw = zero_tma::kConsumerWarps;
     q.tile = uint32_t(t);
     q.off_w = align128(uint64_t(nd) * t * 2);
     q.off_m = q.off_w + align128(4 * t);
@@ -45,19 +48,23 @@ inline zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_
     return q;
 }
 
-inline bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, int *err, zero_tma::Ring *r) {
-    long force_t = 0, force_s = 0, force_g = 0, force_v = 0;
+// max_cw: the most consumer warps the caller has kernels for (8 or 16).
+inline bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, int *err, zero_tma::Ring *r,
+                        uint32_t max_cw = zero_tma::kMaxConsumerWarps) {
+    long force_t = 0, force_s = 0, force_g = 0, force_v = 0, force_c = 0;
     if (const char *e = std::getenv("ZERO_TMA_TILE")) force_t = std::strtol(e, nullptr, 10);
     if (const char *e = std::getenv("ZERO_TMA_STAGES")) force_s = std::strtol(e, nullptr, 10);
     if (const char *e = std::getenv("ZERO_TMA_GROUPS")) force_g = std::strtol(e, nullptr, 10);
     if (const char *e = std::getenv("ZERO_TMA_VW")) force_v = std::strtol(e, nullptr, 10);
+    if (const char *e = std::getenv("ZERO_TMA_CW")) force_c = std::strtol(e, nullptr, 10);
+    const uint32_t cw = (force_c == 16 && max_cw >= 16) ? 16u : uint32_t(zero_tma::kConsumerWarps);
     uint32_t groups, stages, vw;
     uint64_t tile;
     if (force_t >= 256 && force_t % 256 == 0 && force_t <= 16384) {
         tile = uint64_t(force_t);
         groups = force_g == 2 ? 2 : 1;
         stages = force_s >= 2 ? uint32_t(std::min<long>(force_s, zero_tma::kMaxStages)) : zero_tma::kMaxStages;
-        const uint64_t busy = tile * groups / zero_tma::kConsumers;  // keep a group's threads busy
+        const uint64_t busy = tile * groups / (32u * cw);  // keep a group's threads busy
         vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
     } else if (nd <= 2) {
         groups = 2, tile = 2048, stages = 4, vw = 8;
@@ -76,10 +83,17 @@ inline bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, int *err,
     } else {
         return false;
     }
+    if (force_t == 0 && cw > uint32_t(zero_tma::kConsumerWarps)) {
+        // the table's shapes were sized for 8 consumer warps: keep every
+        // thread of a group busy with twice as many
+        const uint64_t busy = tile * groups / (32u * cw);
+        vw = uint32_t(std::min<uint64_t>(vw, busy >= 8 ? 8 : (busy >= 4 ? 4 : 2)));
+    }
     if (force_v == 2 || force_v == 4 || force_v == 8) vw = uint32_t(force_v);
     zero_tma::Ring q = ring_for(nd, tile, 0, groups);
     q.err = err;
     q.vw = vw;
+    q.cw = cw;
     // ZERO_TEST_STALL_PRODUCER=<cta>: that CTA's producer issues nothing, so
     // its consumers' bounded waits run out (tests the ZERO_ETIMEOUT path)
     q.stall_cta = 0xffffffffu;
@@ -127,7 +141,8 @@ inline zero_tma::Ring ring_for_launch(const zero_tma::Ring &r, uint64_t n, uint3
         if (ns < 2 || ns < r.groups * 2) continue;
         q.err = r.err;
         q.stall_cta = r.stall_cta;
-        const uint64_t busy = tile * r.groups / zero_tma::kConsumers;
+        q.cw = r.cw;
+        const uint64_t busy = tile * r.groups / (32u * r.cw);
         q.vw = busy >= 8 ? 8 : (busy >= 4 ? 4 : 2);
         q.stages = uint32_t(ns);
         return q;

@@ -249,12 +249,20 @@ using TmaKernelOf = void (*)(const StepArgs, const zero_tma::Ring, const typenam
 using TmaKernel = TmaKernelOf<zero_tma::kGradRows>;
 using ApplyKernel = TmaKernelOf<zero_tma::kReduced>;
 
-template <bool OM, int SRC = zero_tma::kGradRows>
-TmaKernelOf<SRC> tma_kernel(uint32_t groups, uint32_t vw) {
+template <bool OM, int SRC, int CW>
+TmaKernelOf<SRC> tma_kernel_cw(uint32_t groups, uint32_t vw) {
     using namespace zero_tma;
     if (groups == 2)
-        return vw == 2 ? k_step_tma<OM, 2, 2, SRC> : (vw == 4 ? k_step_tma<OM, 2, 4, SRC> : k_step_tma<OM, 2, 8, SRC>);
-    return vw == 2 ? k_step_tma<OM, 1, 2, SRC> : (vw == 4 ? k_step_tma<OM, 1, 4, SRC> : k_step_tma<OM, 1, 8, SRC>);
+        return vw == 2 ? k_step_tma<OM, 2, 2, SRC, CW>
+                       : (vw == 4 ? k_step_tma<OM, 2, 4, SRC, CW> : k_step_tma<OM, 2, 8, SRC, CW>);
+    return vw == 2 ? k_step_tma<OM, 1, 2, SRC, CW>
+                   : (vw == 4 ? k_step_tma<OM, 1, 4, SRC, CW> : k_step_tma<OM, 1, 8, SRC, CW>);
+}
+
+// ... and x consumer warps (8 or 16; a CTA has 32 + 32 * cw threads)
+template <bool OM, int SRC = zero_tma::kGradRows>
+TmaKernelOf<SRC> tma_kernel(uint32_t groups, uint32_t vw, uint32_t cw = zero_tma::kConsumerWarps) {
+    return cw == 16 ? tma_kernel_cw<OM, SRC, 16>(groups, vw) : tma_kernel_cw<OM, SRC, zero_tma::kConsumerWarps>(groups, vw);
 }
 
 // Launch shapes of the step kernels on one device, computed once per device:
@@ -291,8 +299,9 @@ zero_status_t device_shapes(DeviceShapes *out) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_r, zero_guarded::k_reduce<8, true, true>, kThreads, 0);
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, zero_guarded::k_apply<8, true, true>, kThreads, 0);
-    cudaFuncAttributes fa{};
+    cudaFuncAttributes fa{}, fa16{};
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
+    if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa16, tma_kernel<true>(2, 2, 16));
     DeviceShapes d;
     void *err = nullptr;
     if (e == cudaSuccess) e = cudaGetSymbolAddress(&err, g_wait_error);
@@ -300,15 +309,16 @@ zero_status_t device_shapes(DeviceShapes *out) {
     d.sms = uint32_t(std::max(1, sms));
     d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
     d.grid_guard = std::min(uint32_t(std::max(1, sms) * std::max(1, std::min(occ_r, occ_a))), zero_detail::kMaxSlots);
-    const int64_t budget = int64_t(optin) - int64_t(fa.sharedSizeBytes) - 256;
+    const int64_t budget = int64_t(optin) - int64_t(std::max(fa.sharedSizeBytes, fa16.sharedSizeBytes)) - 256;
     d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
     if (d.tma_smem > 0) {
         for (uint32_t g : {1u, 2u})
-            for (uint32_t vw : {2u, 4u, 8u}) {
-                const void *fs[] = {reinterpret_cast<const void *>(tma_kernel<true>(g, vw)),
-                                    reinterpret_cast<const void *>(tma_kernel<false>(g, vw)),
-                                    reinterpret_cast<const void *>(tma_kernel<true, zero_tma::kReduced>(g, vw)),
-                                    reinterpret_cast<const void *>(tma_kernel<false, zero_tma::kReduced>(g, vw))};
+            for (uint32_t vw : {2u, 4u, 8u})
+            for (uint32_t cw : {8u, 16u}) {
+                const void *fs[] = {reinterpret_cast<const void *>(tma_kernel<true>(g, vw, cw)),
+                                    reinterpret_cast<const void *>(tma_kernel<false>(g, vw, cw)),
+                                    reinterpret_cast<const void *>(tma_kernel<true, zero_tma::kReduced>(g, vw, cw)),
+                                    reinterpret_cast<const void *>(tma_kernel<false, zero_tma::kReduced>(g, vw, cw))};
                 for (const void *f : fs)
                     if (e == cudaSuccess)
                         e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, int(d.tma_smem));
@@ -393,9 +403,9 @@ struct Launcher {
                 const uint64_t tiles = (j1 - j0 + rg.tile - 1) / rg.tile;
                 const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
                 const size_t smem = size_t(rg.stages) * rg.stage_bytes;
-                TmaKernel f = owner_map ? tma_kernel<true>(rg.groups, rg.vw)
-                                        : tma_kernel<false>(rg.groups, rg.vw);
-                launch_ex(f, grid, zero_tma::kThreads, smem, stream, dep, b, rg, zero_tma::NoExtra{});
+                TmaKernel f = owner_map ? tma_kernel<true>(rg.groups, rg.vw, rg.cw)
+                                        : tma_kernel<false>(rg.groups, rg.vw, rg.cw);
+                launch_ex(f, grid, 32 + 32 * rg.cw, smem, stream, dep, b, rg, zero_tma::NoExtra{});
             } else if (vec) {
                 const bool rb8 = ldg_rows(b.nd) == 8;
                 auto f = owner_map ? (rb8 ? k_step_vec8<true, 8, kMinB> : k_step_vec8<true, kRB, kMinB>)
@@ -758,9 +768,9 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
                 const zero_tma::Ring rg = ring_for_launch(ring, j1 - j0, 2, shapes.sms, shapes.tma_smem);
                 const uint64_t tiles = (j1 - j0 + rg.tile - 1) / rg.tile;
                 const uint32_t g = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
-                ApplyKernel f = om ? tma_kernel<true, zero_tma::kReduced>(rg.groups, rg.vw)
-                                   : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw);
-                launch_ex(f, g, zero_tma::kThreads, size_t(rg.stages) * rg.stage_bytes, stream, dep, y, rg,
+                ApplyKernel f = om ? tma_kernel<true, zero_tma::kReduced>(rg.groups, rg.vw, rg.cw)
+                                   : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw, rg.cw);
+                launch_ex(f, g, 32 + 32 * rg.cw, size_t(rg.stages) * rg.stage_bytes, stream, dep, y, rg,
                           zero_tma::ApplyExtra{gw});
             } else {
                 auto f = vec ? (w32 ? (om ? zero_guarded::k_apply<8, true, true> : zero_guarded::k_apply<8, false, true>)

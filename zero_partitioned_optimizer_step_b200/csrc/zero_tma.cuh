@@ -5,7 +5,7 @@
 // Warp 0 is the producer.  Per tile of `tile` elements it issues one
 // cp.async.bulk per gradient row (Nd rows, spread over its lanes) and one per
 // state array and owner segment, all completing on the stage's `full`
-// mbarrier.  Warps 1..8 are consumers: they read the stage from shared memory,
+// mbarrier.  Warps 1..CW are consumers (CW = 8 or 16, a template parameter): they read the stage from shared memory,
 // sum the rows in rank order, run Adam, and write w, m, v and the bf16
 // parameters (every replica row, or the owner shard) straight from registers
 // with 16-byte streaming stores.  The stage is released through its `empty`
@@ -33,9 +33,12 @@ namespace zero_tma {
 using zero_dev::AdamConsts;
 using zero_dev::StepArgs;
 
+// Consumer warps: 8 by default (kThreads = 288 threads per CTA), or 16 (544),
+// the kernel's CW template parameter; the ring records which.
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumers = 32 * kConsumerWarps;
 constexpr int kThreads = 32 + kConsumers;  // warp 0 produces
+constexpr int kMaxConsumerWarps = 16;
 // Consumers form GROUPS groups (a template parameter, 1 or 2) that take the
 // CTA's tiles in turn.  Tile k goes to stage k % stages and to group
 // k % GROUPS; the host makes `stages` a multiple of GROUPS, so every stage
@@ -56,6 +59,7 @@ struct Ring {
     uint32_t stall_cta;  // test of the bounded waits: this CTA's producer issues
                          // nothing (0xffffffff: none)
     uint32_t vw;
+    uint32_t cw;         // consumer warps the kernel was instantiated with
     uint32_t tile;
     uint32_t stages;  // a multiple of groups
     uint32_t groups;  // consumer groups the kernel was instantiated with
@@ -276,17 +280,18 @@ __device__ __forceinline__ void stg_bf16_ptrs(uint16_t *const *rows, uint64_t of
     }
 }
 
-template <bool OWNER_MAP, int GROUPS, int VW, int SRC = kGradRows>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool OWNER_MAP, int GROUPS, int VW, int SRC = kGradRows, int CW = kConsumerWarps>
+__global__ void __launch_bounds__(32 + 32 * CW, 1)
     k_step_tma(const StepArgs a, const Ring ring, const typename ExtraOf<SRC>::type x) {
-    constexpr uint32_t kGroupThreads = kConsumers / GROUPS;
+    constexpr uint32_t kCons = 32u * CW;
+    constexpr uint32_t kGroupThreads = kCons / GROUPS;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kMaxStages];
     __shared__ __align__(8) uint64_t empty_bar[kMaxStages];
     __shared__ uint64_t stage_tile[kMaxStages];  // tile a stage was filled with
     __shared__ int s_abort;
-    __shared__ double s_norm[kConsumerWarps];
-    __shared__ uint32_t s_bad[kConsumerWarps];
+    __shared__ double s_norm[CW];
+    __shared__ uint32_t s_bad[CW];
     __shared__ const uint16_t *s_rows[SRC == kPeerRows ? zero_dev::kMaxPeers : 1];
     __shared__ uint16_t *s_prow[SRC == kPeerRows ? zero_dev::kMaxPeers : 1];
 
@@ -314,8 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_barrier_init();
     }
     if constexpr (SRC == kPeerRows) {
-        for (uint32_t i = threadIdx.x; i < a.nd; i += kThreads) s_rows[i] = x.g[i];
-        for (uint32_t i = threadIdx.x; i < a.n_prow; i += kThreads) s_prow[i] = x.p[i];
+        for (uint32_t i = threadIdx.x; i < a.nd; i += blockDim.x) s_rows[i] = x.g[i];
+        for (uint32_t i = threadIdx.x; i < a.n_prow; i += blockDim.x) s_prow[i] = x.p[i];
     }
     __syncthreads();
     volatile int *abort_flag = &s_abort;
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (SRC == kPeerRows) {
         // every consumer's peer stores are performed before the kernel
         // completes: a consumer barrier, then one cumulative system fence
-        barrier_or(1 + GROUPS, kConsumers, false);
+        barrier_or(1 + GROUPS, kCons, false);
         if (ct == 0) __threadfence_system();
     }
     zero_dev::pdl_wait();  // predecessor done: its norm slots are final
@@ -461,11 +466,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             s_norm[warp - 1] = acc;
             s_bad[warp - 1] = bad;
         }
-        barrier_or(1 + GROUPS, kConsumers, false);
+        barrier_or(1 + GROUPS, kCons, false);
         if (ct == 0) {
             double t = 0.0;
             uint32_t b = 0;
-            for (int i = 0; i < kConsumerWarps; ++i) {
+            for (int i = 0; i < CW; ++i) {
                 t += s_norm[i];
                 b += s_bad[i];
             }
