@@ -607,6 +607,20 @@ def guarded_launches(lp):
     return 2 * n + 1
 
 
+def second_pass_kernel(wl):
+    """The kernel zero_step_guarded runs its second pass in (aligned bodies):
+    the bulk-copy ring where the parameters are written once (stage 3),
+    else k_apply_bulk (replica rows as bulk copies from shared memory), or
+    k_apply under ZERO_GUARD_APPLY=ldst; ZERO_STEP_KERNEL=tma forces the
+    ring."""
+    forced = os.environ.get("ZERO_STEP_KERNEL", "")
+    if forced == "tma" or (forced != "ldg" and not wl.replicas):
+        return "k_step_tma"
+    if not wl.replicas:
+        return "k_apply"
+    return "k_apply" if os.environ.get("ZERO_GUARD_APPLY") == "ldst" else "k_apply_bulk"
+
+
 def run_guarded(args, cfg, rank, world, dist):
     """--guarded: the two-pass step with global-norm clipping (at
     --max-grad-norm) and skipping on non-finite gradients, zero_step_guarded,
@@ -680,7 +694,7 @@ def run_guarded(args, cfg, rank, world, dist):
                    "hbm_bytes_per_step": step_bytes,
                    "l2": "inputs larger than L2 (%.2f GB touched per step); no flush" % (step_bytes / 1e9)},
         "hbm_gbs": step_bytes / (elapsed / args.steps) / 1e9,
-        "roofline": {"kernel": "guarded step (k_reduce, k_guard_finalize, k_apply: the whole call)",
+        "roofline": {"kernel": "guarded step (k_reduce, k_guard_finalize, %s: the whole call)" % second_pass_kernel(wl),
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind + " (copy bandwidth)",
                      "traffic": None, "algorithmic_bytes_per_call": g_bytes,

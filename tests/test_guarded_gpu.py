@@ -32,13 +32,27 @@ def test_adamw_fused_bit_exact(kernel, psi, nd, stage, units, monkeypatch):
         assert all(v == 0 for v in diff.values()), diff
 
 
-@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+def _second_pass(kernel, monkeypatch):
+    """tma: the second pass in the bulk-copy ring kernel; ldg: in the
+    16-byte-load kernels, with bulk replica copies (k_apply_bulk) where there
+    are replica rows; ldst: k_apply with per-thread replica stores; tma16:
+    the ring kernel with 16 consumer warps."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", "ldg" if kernel == "ldst" else kernel[:3])
+    if kernel == "ldst":
+        monkeypatch.setenv("ZERO_GUARD_APPLY", "ldst")
+    if kernel == "tma16":
+        monkeypatch.setenv("ZERO_TMA_CW", "16")
+
+
+@pytest.mark.parametrize("kernel", ["tma", "ldg", "ldst"])
 @pytest.mark.parametrize("psi,nd,stage,units,align", [
-    (500_000, 8, 2, None, 64), (300_001, 16, 3, [100_000, 3, 199_998], 64), (77_777, 5, 1, None, 1)])
+    (500_000, 8, 2, None, 64), (300_001, 16, 3, [100_000, 3, 199_998], 64), (77_777, 5, 1, None, 1),
+    (600_000, 6, 2, [200_000, 8, 399_992], 8)])
 def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align, kernel, monkeypatch):
-    """A guard that never triggers gives the fused step's bits (second pass
-    in the bulk-copy kernel, or in the 16-byte-load kernel)."""
-    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
+    """A guard that never triggers gives the fused step's bits, whichever
+    kernel runs the second pass (several units at stage 2: replicas with an
+    owner map)."""
+    _second_pass(kernel, monkeypatch)
     a = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
     b = Case(psi, nd, stage, 1 << 15, units=units, align=align, config_id=13, adam=ADAMW)
     for t in (1, 2):
@@ -51,14 +65,12 @@ def test_guarded_without_trigger_equals_fused(psi, nd, stage, units, align, kern
         assert torch.equal(a.params.view(torch.int16), b.params.view(torch.int16))
 
 
-@pytest.mark.parametrize("kernel", ["tma", "ldg", "tma16"])
+@pytest.mark.parametrize("kernel", ["tma", "ldg", "ldst", "tma16"])
 @pytest.mark.parametrize("psi,nd,stage,units", [(500_000, 8, 2, None),
-                                                (300_001, 16, 3, [100_000, 3, 199_998])])
+                                                (300_001, 16, 3, [100_000, 3, 199_998]),
+                                                (1_000_001, 3, 2, None)])
 def test_guarded_clipping(psi, nd, stage, units, kernel, monkeypatch):
-    """tma16: the second pass in the bulk-copy kernel with 16 consumer warps."""
-    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel[:3])
-    if kernel == "tma16":
-        monkeypatch.setenv("ZERO_TMA_CW", "16")
+    _second_pass(kernel, monkeypatch)
     c = Case(psi, nd, stage, 1 << 15, units=units, sigma=1e-2, config_id=14, adam=ADAMW)
     for t in (1, 2, 3):
         diff, coef, skipped = c.guarded_step_and_compare(t, 0.05, True)
@@ -94,10 +106,12 @@ def test_guarded_requires_its_buffers():
                             overflow=c.ovf, workspace=c.ws)
 
 
+@pytest.mark.parametrize("apply", ["bulk", "ldst"])
 @pytest.mark.parametrize("offset", [0, 4])
-def test_guarded_state_at_16_byte_offsets(offset):
+def test_guarded_state_at_16_byte_offsets(offset, apply, monkeypatch):
     """The fp32 arrays 32-byte aligned (32-byte accesses) or only 16-byte
     aligned (16-byte accesses): the same bits."""
+    monkeypatch.setenv("ZERO_GUARD_APPLY", apply)
     psi, nd = 500_000, 8
     c = Case(psi, nd, 2, 1 << 15, config_id=15, adam=ADAMW)
     for name in ("w", "m", "v", "red"):

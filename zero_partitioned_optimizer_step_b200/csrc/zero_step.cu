@@ -274,6 +274,7 @@ struct DeviceShapes {
     int *err = nullptr;       // g_wait_error on this device
     uint32_t grid_ldg = 0;
     uint32_t grid_guard = 0;  // the guarded step's two passes (fewer registers)
+    uint32_t grid_apply_bulk = 0;  // the guarded step's second pass with bulk replica copies
     uint32_t sms = 0;
     uint32_t tma_smem = 0;
 };
@@ -290,7 +291,7 @@ zero_status_t device_shapes(DeviceShapes *out) {
         *out = it->second;
         return ZERO_OK;
     }
-    int sms = 0, occ = 0, optin = 0, occ_r = 0, occ_a = 0;
+    int sms = 0, occ = 0, optin = 0, occ_r = 0, occ_a = 0, occ_b = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     if (e == cudaSuccess)
@@ -299,6 +300,8 @@ zero_status_t device_shapes(DeviceShapes *out) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_r, zero_guarded::k_reduce<8, true, true>, kThreads, 0);
     if (e == cudaSuccess)
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, zero_guarded::k_apply<8, true, true>, kThreads, 0);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, zero_guarded::k_apply_bulk<true, true>, kThreads, 0);
     cudaFuncAttributes fa{}, fa16{};
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, tma_kernel<true>(2, 2));
     if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa16, tma_kernel<true>(2, 2, 16));
@@ -309,6 +312,13 @@ zero_status_t device_shapes(DeviceShapes *out) {
     d.sms = uint32_t(std::max(1, sms));
     d.grid_ldg = std::min(uint32_t(std::max(1, sms) * std::max(1, occ)), zero_detail::kMaxSlots);
     d.grid_guard = std::min(uint32_t(std::max(1, sms) * std::max(1, std::min(occ_r, occ_a))), zero_detail::kMaxSlots);
+    // three CTAs per SM (24 warps): the pass is bound by load latency
+    // (long-scoreboard stalls) at two; measured on B200 with the guarded
+    // GPT-2-small step, 1 / 2 / 3 / 4 CTAs per SM gave 5.78 / 6.02 / 6.23 /
+    // 5.99 TB/s; ZERO_APPLY_BULK_CTAS overrides (tuning)
+    int per_sm = 3;
+    if (const char *v = std::getenv("ZERO_APPLY_BULK_CTAS")) per_sm = std::max(1, std::atoi(v));
+    d.grid_apply_bulk = uint32_t(std::max(1, sms) * std::max(1, std::min(occ_b, per_sm)));
     const int64_t budget = int64_t(optin) - int64_t(std::max(fa.sharedSizeBytes, fa16.sharedSizeBytes)) - 256;
     d.tma_smem = budget > 0 ? uint32_t(budget) : 0;
     if (d.tma_smem > 0) {
@@ -753,6 +763,11 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     const int choice = kernel_choice();
     const bool tma = (choice == 2 || (choice == 0 && a.n_prow == 1)) &&
                      choose_ring(2, false, shapes.tma_smem, shapes.err, &ring);
+    // With replica rows, the vector body's parameters go out as bulk copies
+    // from shared memory (k_apply_bulk) unless ZERO_GUARD_APPLY=ldst asks for
+    // k_apply's per-thread stores.
+    const char *ga = std::getenv("ZERO_GUARD_APPLY");
+    const bool bulk_replicas = a.n_prow > 1 && !(ga && std::strcmp(ga, "ldst") == 0);
     a.ws_mode = 0;
     for (uint64_t bk = 0; bk < p->n_buckets; ++bk) {
         StepArgs x;
@@ -772,6 +787,11 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
                                    : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw, rg.cw);
                 launch_ex(f, g, 32 + 32 * rg.cw, size_t(rg.stages) * rg.stage_bytes, stream, dep, y, rg,
                           zero_tma::ApplyExtra{gw});
+            } else if (vec && bulk_replicas) {
+                auto f = w32 ? (om ? zero_guarded::k_apply_bulk<true, true> : zero_guarded::k_apply_bulk<false, true>)
+                             : (om ? zero_guarded::k_apply_bulk<true, false> : zero_guarded::k_apply_bulk<false, false>);
+                launch_ex(f, shapes.grid_apply_bulk, kThreads, 0, stream, dep, y,
+                          static_cast<const zero_guarded::GuardWord *>(gw));
             } else {
                 auto f = vec ? (w32 ? (om ? zero_guarded::k_apply<8, true, true> : zero_guarded::k_apply<8, false, true>)
                                     : (om ? zero_guarded::k_apply<8, true> : zero_guarded::k_apply<8, false>))
