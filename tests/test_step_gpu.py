@@ -126,6 +126,26 @@ def test_norm_and_overflow_flag(kernel):
     assert int(c.ovf.item()) == 0
 
 
+@pytest.mark.parametrize("scale", [1e22, 1e-22, "mixed"])
+def test_norm_at_extreme_magnitudes(scale, kernel):
+    """Reduced gradients whose squares leave the fp32 range: all of them
+    (|g_sum| near 1e19, squares past fp32's maximum; |g_sum| near 1e-25,
+    squares below its smallest subnormal), or one column in 16 scaled up
+    among ordinary values.  The norm is a double-precision sum of squares,
+    so it must match the oracle's and stay finite: a square taken in fp32
+    would overflow or vanish here."""
+    c = Case(100_000, 4, 2, 30_000, config_id=7)
+    G = c.grads(1).float()
+    if scale == "mixed":
+        G[:, ::16] *= 1e22
+    else:
+        G *= scale
+    G = G.to(torch.bfloat16)
+    c.step_and_compare(1, G)
+    n = c.norm.item()
+    assert np.isfinite(n) and n > 0 and int(c.ovf.item()) == 0
+
+
 def test_norm_is_deterministic(kernel):
     c = Case(300_000, 8, 2, 30_000, config_id=6, with_reduced=False)
     G = c.grads(1)
