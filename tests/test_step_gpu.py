@@ -270,3 +270,20 @@ def test_bulk_kernel_vector_widths(cw, vw, psi, nd, stage, units, owner, monkeyp
     for t in (1, 2):
         diff = c.step_and_compare(t)
         assert all(v == 0 for v in diff.values()), diff
+
+
+@pytest.mark.parametrize("vw", ["2", "4", "8"])
+@pytest.mark.parametrize("psi,nd,units,bucket", [
+    (700_001, 8, None, 1 << 18), (300_007, 2, None, 1 << 18), (500_000, 64, None, 1 << 18),
+    (600_000, 6, [200_000, 8, 399_992], 1 << 16), (50_000, 16, None, 4096)])
+def test_bulk_kernel_replica_rows_as_bulk_copies(vw, psi, nd, units, bucket, monkeypatch):
+    """The bulk-copy kernel with its replica rows written as 1-D bulk copies
+    from shared memory (ZERO_TMA_BULKP=1), stage 2: the same bits as the
+    oracle (several units: an owner map; small buckets: the cut ring)."""
+    monkeypatch.setenv("ZERO_STEP_KERNEL", "tma")
+    monkeypatch.setenv("ZERO_TMA_VW", vw)
+    monkeypatch.setenv("ZERO_TMA_BULKP", "1")
+    c = Case(psi, nd, 2, bucket, units=units, align=8 if units else 64, config_id=17)
+    for t in (1, 2):
+        diff = c.step_and_compare(t)
+        assert all(v == 0 for v in diff.values()), diff

@@ -420,6 +420,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
     const bool tma = (choice == 2 || (choice == 0 && !replicas)) &&
                      zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring,
                                             zero_tma::kConsumerWarps);
+    ring.bulk_p = 0;  // the peer rows are stored through their pointers
     // Vector launches after the first of the call overlap their predecessor
     // (programmatic dependent launch): consecutive launches of one call share
     // only the norm slots, which every kernel adds to after its predecessor
@@ -455,7 +456,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
             const uint64_t tiles = (p1 - p0 + rg.tile - 1) / rg.tile;
             const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
             launch_pdl(peer_tma_kernel(rg.groups, rg.vw), grid, zero_tma::kThreads,
-                       size_t(rg.stages) * rg.stage_bytes, stream, dep, sa, rg, tab);
+                       zero_ring::ring_smem_bytes(rg), stream, dep, sa, rg, tab);
         } else if (vec) {
             launch_pdl(k_step_peer, shapes.grid, kThreads, 0, stream, dep, x, tab);
         } else {

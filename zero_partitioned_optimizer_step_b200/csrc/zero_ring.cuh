@@ -35,6 +35,12 @@ inline uint32_t align128(uint64_t x) { return uint32_t((x + 127) & ~uint64_t(127
 // work).  ZERO_TMA_TILE / ZERO_TMA_STAGES / ZERO_TMA_GROUPS / ZERO_TMA_VW override the
 // shape (tuning; a tile must be a positive multiple of 256).  `err` is the
 // device error word the kernel's bounded waits report to.
+// Dynamic shared memory of a launch: the stages, then (bulk_p) two
+// parameter tiles per consumer group.
+inline size_t ring_smem_bytes(const zero_tma::Ring &r) {
+    return size_t(r.stages) * r.stage_bytes + (r.bulk_p ? size_t(r.groups) * 2 * r.tile * 2 : 0);
+}
+
 inline zero_tma::Ring ring_for(uint32_t nd, uint64_t t, uint32_t stages, uint32_t groups) {
     zero_tma::Ring q{};
     q.cw = zero_tma::kConsumerWarps;
@@ -102,7 +108,17 @@ inline bool choose_ring(uint32_t nd, bool read_heavy, uint32_t budget, int *err,
         const unsigned long v = std::strtoul(e, &end, 10);
         if (end != e && v < 0xffffffffu) q.stall_cta = uint32_t(v);
     }
-    uint64_t ns = std::min<uint64_t>(budget / q.stage_bytes, stages);
+    // Replica rows as bulk copies from shared memory at Nd <= 2, where a
+    // tile's copies are few and large (2 per tile of 4 KB each): K1 went from
+    // 0.950 to 0.979 of copy bandwidth at Nd = 2 (64 MB buckets, 5e8
+    // params), was flat at Nd = 4, and lost 6 %, 3 % and 30 % at Nd = 8, 16
+    // and 64, where one thread issues Nd small copies per tile.
+    // ZERO_TMA_BULKP=0|1 overrides.
+    q.bulk_p = (!read_heavy && nd <= 2) ? 1u : 0u;
+    if (const char *e = std::getenv("ZERO_TMA_BULKP")) q.bulk_p = e[0] == '1' ? 1u : 0u;
+    const uint64_t pbytes = q.bulk_p ? uint64_t(groups) * 2 * tile * 2 : 0;
+    if (pbytes >= budget) return false;
+    uint64_t ns = std::min<uint64_t>((budget - pbytes) / q.stage_bytes, stages);
     ns -= ns % groups;  // every stage belongs to one group
     if (ns < 2) return false;
     q.stages = uint32_t(ns);
@@ -136,7 +152,10 @@ inline zero_tma::Ring ring_for_launch(const zero_tma::Ring &r, uint64_t n, uint3
     const uint64_t half = budget / 2 - 1024;  // room for a second CTA's ring and static shared memory
     for (uint64_t tile = r.tile; tile >= 512; tile /= 2) {
         zero_tma::Ring q = ring_for(nd, tile, 0, r.groups);
-        uint64_t ns = std::min<uint64_t>(half / q.stage_bytes, zero_tma::kMaxStages);
+        q.bulk_p = r.bulk_p;
+        const uint64_t pbytes = q.bulk_p ? uint64_t(r.groups) * 2 * tile * 2 : 0;
+        if (pbytes >= half) continue;
+        uint64_t ns = std::min<uint64_t>((half - pbytes) / q.stage_bytes, zero_tma::kMaxStages);
         ns -= ns % r.groups;
         if (ns < 2 || ns < r.groups * 2) continue;
         q.err = r.err;

@@ -412,7 +412,7 @@ struct Launcher {
                 const zero_tma::Ring rg = ring_for_launch(ring, j1 - j0, b.nd, shapes.sms, shapes.tma_smem);
                 const uint64_t tiles = (j1 - j0 + rg.tile - 1) / rg.tile;
                 const uint32_t grid = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
-                const size_t smem = size_t(rg.stages) * rg.stage_bytes;
+                const size_t smem = zero_ring::ring_smem_bytes(rg);
                 TmaKernel f = owner_map ? tma_kernel<true>(rg.groups, rg.vw, rg.cw)
                                         : tma_kernel<false>(rg.groups, rg.vw, rg.cw);
                 launch_ex(f, grid, 32 + 32 * rg.cw, smem, stream, dep, b, rg, zero_tma::NoExtra{});
@@ -763,6 +763,7 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
     const int choice = kernel_choice();
     const bool tma = (choice == 2 || (choice == 0 && a.n_prow == 1)) &&
                      choose_ring(2, false, shapes.tma_smem, shapes.err, &ring);
+    ring.bulk_p = 0;  // this pass's parameters: per-thread stores
     // With replica rows, the vector body's parameters go out as bulk copies
     // from shared memory (k_apply_bulk) unless ZERO_GUARD_APPLY=ldst asks for
     // k_apply's per-thread stores.
@@ -785,7 +786,7 @@ ZERO_API zero_status_t zero_step_guarded(const zero_plan_t *p, const zero_bufs_t
                 const uint32_t g = uint32_t(std::min<uint64_t>(tiles, shapes.sms));
                 ApplyKernel f = om ? tma_kernel<true, zero_tma::kReduced>(rg.groups, rg.vw, rg.cw)
                                    : tma_kernel<false, zero_tma::kReduced>(rg.groups, rg.vw, rg.cw);
-                launch_ex(f, g, 32 + 32 * rg.cw, size_t(rg.stages) * rg.stage_bytes, stream, dep, y, rg,
+                launch_ex(f, g, 32 + 32 * rg.cw, zero_ring::ring_smem_bytes(rg), stream, dep, y, rg,
                           zero_tma::ApplyExtra{gw});
             } else if (vec && bulk_replicas) {
                 auto f = w32 ? (om ? zero_guarded::k_apply_bulk<true, true> : zero_guarded::k_apply_bulk<false, true>)

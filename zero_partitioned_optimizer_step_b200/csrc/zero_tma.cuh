@@ -64,6 +64,9 @@ struct Ring {
     uint32_t stages;  // a multiple of groups
     uint32_t groups;  // consumer groups the kernel was instantiated with
     uint32_t stage_bytes;
+    uint32_t bulk_p;  // 1: with replica rows (fused step), the bf16 parameters
+                      // go to two shared-memory tiles per group after the
+                      // stages and out as one 1-D bulk copy per row and tile
     uint32_t off_w, off_m, off_v;
 };
 
@@ -262,6 +265,27 @@ struct ExtraOf<kPeerRows> {
     using type = zero_dev::PeerTable;
 };
 
+// bf16(w) of VW elements into a shared-memory tile
+template <int VW>
+__device__ __forceinline__ void sts_bf16(uint16_t *p, const float w[VW]) {
+    uint32_t pk[VW / 2];
+#pragma unroll
+    for (int h = 0; h < VW / 2; ++h) pk[h] = zero_dev::pack_bf16x2(w[2 * h], w[2 * h + 1]);
+    if constexpr (VW == 2) {
+        *reinterpret_cast<uint32_t *>(p) = pk[0];
+    } else if constexpr (VW == 4) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pk[0], pk[1]);
+    } else {
+        *reinterpret_cast<uint4 *>(p) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+}
+
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // bf16(w) of VW elements to `rows` parameter rows given by pointer
 template <int VW>
 __device__ __forceinline__ void stg_bf16_ptrs(uint16_t *const *rows, uint64_t off, const float w[VW], uint32_t n) {
@@ -388,6 +412,14 @@ __global__ void __launch_bounds__(32 + 32 * CW, 1)
     const uint32_t gt = uint32_t(ct) % kGroupThreads;
     double acc = 0.0;
     uint32_t bad = 0;
+    // Replica rows as bulk copies (ring.bulk_p): the group's two tiles of
+    // parameters alternate; at the end of a tile the issuing thread (gt 0)
+    // waits until the previous tile's copies have read the other one, the
+    // group's barrier publishes that and this tile's writes, and then it
+    // issues one copy per replica row.
+    const bool bulkp = SRC == kGradRows && ring.bulk_p && a.n_prow > 1;
+    uint16_t *ptile = reinterpret_cast<uint16_t *>(smem + size_t(NS) * ring.stage_bytes) + size_t(grp) * 2 * T;
+    uint32_t pb = 0;
     uint32_t k = grp;
     for (uint64_t tile = blockIdx.x + uint64_t(grp) * gridDim.x; tile < n_tiles;
          tile += uint64_t(GROUPS) * gridDim.x, k += GROUPS) {
@@ -440,14 +472,29 @@ __global__ void __launch_bounds__(32 + 32 * CW, 1)
                 stg_f32<VW>(a.m + si, mv);
                 stg_f32<VW>(a.v + si, vq);
                 if constexpr (SRC == kPeerRows) stg_bf16_ptrs<VW>(s_prow, pi, wv, a.n_prow);
+                else if (bulkp) sts_bf16<VW>(ptile + size_t(pb) * T + size_t(vv) * VW, wv);
                 else stg_bf16_rows<VW>(a.params + pi, wv, a.n_prow, a.param_stride);
             }
+        }
+        if (bulkp) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // this thread's tile writes
+            if (gt == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
         // the whole group has read the stage (or the CTA is giving up): same
         // decision in all of its threads, then hand the stage back
         if (barrier_or(1 + grp, kGroupThreads, failed || *abort_flag)) break;
+        if (bulkp && gt == 0) {
+            // replica rows are contiguous in logical order (no owner jump)
+            uint16_t *row = a.params + uint64_t(a.p_base + int64_t(jb));
+            for (uint32_t r = 0; r < a.n_prow; ++r)
+                bulk_store(row + uint64_t(r) * a.param_stride, ptile + size_t(pb) * T, n * 2u);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        pb ^= 1u;
         if (gt == 0) mbar_arrive(&empty_bar[s]);
     }
+    // the parameter tiles must outlive their copies, which also complete the writes
+    if (bulkp && gt == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 
     if constexpr (SRC == kPeerRows) {
         // every consumer's peer stores are performed before the kernel
