@@ -68,6 +68,8 @@ SHAPES = [
     (250_001, 64, 2, 1 << 14, 64, None, -1),
     (1_000_000, 64, 2, 100_000, 64, None, 63),
     (300_001, 16, 3, 20_000, 64, [100_000, 1, 200_000], 9),
+    (77_777, 2, 2, 10_000, 8, None, -1),            # replica rows as bulk copies, ragged tail
+    (90_001, 2, 1, 4096, 8, [30_000, 60_001], -1),  # the same, small buckets (cut ring), two units
 ]
 
 
@@ -144,3 +146,31 @@ def test_random_shapes_match_oracle(seed, monkeypatch):
         for t in (1, 2):
             diff = c.step_and_compare(t)
             assert all(v == 0 for v in diff.values()), (kernel, diff)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_guarded_shapes_match_oracle(seed, monkeypatch):
+    """The guarded step on seeded random plans (all ranks' view), with a clip
+    threshold that clips, one that does not, or none, through every kernel
+    its second pass can take: the bulk-copy ring (ZERO_STEP_KERNEL=tma), the
+    replica rows as bulk copies from shared memory (ldg), and per-thread
+    stores (ldst)."""
+    rnd = random.Random(5000 + seed)
+    psi, nd, stage, bucket, align, units, _ = _random_case(rnd)
+    stage = max(stage, 1)   # the oracle's guarded step is the partitioned one
+    bucket = max(bucket, 1000)   # two passes of 7-element buckets: too many launches for a test
+    max_norm = rnd.choice([0.0, 1e-4, 1e-4, 1e9])
+    for second in ("tma", "ldg", "ldst"):
+        monkeypatch.setenv("ZERO_STEP_KERNEL", "ldg" if second == "ldst" else second)
+        if second == "ldst":
+            monkeypatch.setenv("ZERO_GUARD_APPLY", "ldst")
+        else:
+            monkeypatch.delenv("ZERO_GUARD_APPLY", raising=False)
+        c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=60 + seed)
+        for t in (1, 2):
+            diff, coef, skipped = c.guarded_step_and_compare(t, max_norm, True)   # tolerances
+            assert not skipped
+            if max_norm == 1e-4:
+                assert coef < 1
+            else:   # no clipping: the same bits as the definition
+                assert coef == 1 and all(v == 0 for v in diff.values()), (second, diff)
