@@ -146,6 +146,25 @@ def test_norm_at_extreme_magnitudes(scale, kernel):
     assert np.isfinite(n) and n > 0 and int(c.ovf.item()) == 0
 
 
+def test_subnormal_gradients(kernel):
+    """bf16 subnormal gradients (exponent field 0): their fp32 sums, the
+    gradient Adam sees and the first moment are fp32 subnormals, and the
+    second moment underflows to zero.  Every operation must keep subnormals
+    as IEEE arithmetic does (no flush to zero), packed pairs included."""
+    c = Case(50_000, 4, 2, 16_384, config_id=8)
+    gen = torch.Generator(device="cuda").manual_seed(8)
+    n = c.op.psi_pad
+    mant = torch.randint(1, 128, (4, n), generator=gen, device="cuda", dtype=torch.int32)
+    sign = torch.randint(0, 2, (4, n), generator=gen, device="cuda", dtype=torch.int32) << 15
+    G = (mant | sign).to(torch.int16).view(torch.bfloat16)
+    G[:, 50_000:] = 0                     # padding
+    for t in (1, 2):
+        diff = c.step_and_compare(t, G)
+        assert all(v == 0 for v in diff.values()), diff
+    m = f32(c.m)[:50_000]
+    assert np.count_nonzero((m != 0) & (np.abs(m) < np.finfo(np.float32).tiny)) > 1000
+
+
 def test_norm_is_deterministic(kernel):
     c = Case(300_000, 8, 2, 30_000, config_id=6, with_reduced=False)
     G = c.grads(1)

@@ -121,6 +121,34 @@ __device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w
     adam1c(g_sum, 1.0f, c, w, m, v);
 }
 
+// ---------------------------------------------------------------------------
+// Two fp32 lanes in one 64-bit register, for sm_100's packed fp32 add (one
+// instruction per pair; each lane rounded to nearest exactly as the scalar
+// add).  Used for the rank-order sum only, a chain of adds of loaded values.
+// The multiplications and additions of the Adam update stay scalar
+// (__fmul_rn / __fadd_rn, never contracted): measured on B200 against them,
+// packed multiplies and adds each matched bit for bit alone, but a packed
+// multiply feeding a packed add differed in 19 % of pairs, as if fused into
+// one rounding -- and so did the same pair written as packed fused
+// multiply-adds with a -0 or 1 operand, once the constants were run-time
+// values.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// Two bf16 (one 32-bit word, low half first) as an fp32 pair: exact.
+__device__ __forceinline__ uint64_t f2_bf16x2(uint32_t w) { return f2_pack(bf16lo(w), bf16hi(w)); }
+
 // Per-CTA partials of the gradient-norm / overflow reduction, added to slot
 // blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
 // so the reported norm is the same on every run of the same launch shapes.

@@ -194,6 +194,24 @@ __device__ __forceinline__ void lds_bf16(const unsigned char *p, float f[VW]) {
     }
 }
 
+// VW bf16 from shared memory as VW / 2 fp32 pairs (exact).
+template <int VW>
+__device__ __forceinline__ void lds_bf16x2(const unsigned char *p, uint64_t f[VW / 2]) {
+    if constexpr (VW == 2) {
+        f[0] = zero_dev::f2_bf16x2(*reinterpret_cast<const uint32_t *>(p));
+    } else if constexpr (VW == 4) {
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        f[0] = zero_dev::f2_bf16x2(x.x);
+        f[1] = zero_dev::f2_bf16x2(x.y);
+    } else {
+        const uint4 x = *reinterpret_cast<const uint4 *>(p);
+        f[0] = zero_dev::f2_bf16x2(x.x);
+        f[1] = zero_dev::f2_bf16x2(x.y);
+        f[2] = zero_dev::f2_bf16x2(x.z);
+        f[3] = zero_dev::f2_bf16x2(x.w);
+    }
+}
+
 template <int VW>
 __device__ __forceinline__ void lds_f32(const unsigned char *p, float f[VW]) {
     if constexpr (VW == 2) {
@@ -436,19 +454,23 @@ __global__ void __launch_bounds__(32 + 32 * CW, 1)
         if (!failed) {
             const uint32_t nv = n / VW;
             for (uint32_t vv = gt; vv < nv; vv += kGroupThreads) {
+                // the rank-order sum, in fp32 pairs (each lane rounded as a
+                // scalar add would be)
                 float sum[VW];
                 if constexpr (SRC == kReduced) {
                     lds_f32<VW>(st + size_t(vv) * (4 * VW), sum);
                 } else {
                     const unsigned char *gp = st + size_t(vv) * (2 * VW);
-                    float f[VW];
-                    lds_bf16<VW>(gp, sum);
+                    uint64_t s2[VW / 2], f2[VW / 2];
+                    lds_bf16x2<VW>(gp, s2);
 #pragma unroll 4
                     for (uint32_t r = 1; r < a.nd; ++r) {
-                        lds_bf16<VW>(gp + size_t(r) * T * 2, f);
+                        lds_bf16x2<VW>(gp + size_t(r) * T * 2, f2);
 #pragma unroll
-                        for (int e = 0; e < VW; ++e) sum[e] = __fadd_rn(sum[e], f[e]);
+                        for (int h = 0; h < VW / 2; ++h) s2[h] = zero_dev::f2_add(s2[h], f2[h]);
                     }
+#pragma unroll
+                    for (int h = 0; h < VW / 2; ++h) zero_dev::f2_unpack(s2[h], sum[2 * h], sum[2 * h + 1]);
                 }
                 float wv[VW], mv[VW], vq[VW];
                 lds_f32<VW>(st + ring.off_w + size_t(vv) * (4 * VW), wv);
