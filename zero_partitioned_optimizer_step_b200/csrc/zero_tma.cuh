@@ -322,8 +322,14 @@ __device__ __forceinline__ void stg_bf16_ptrs(uint16_t *const *rows, uint64_t of
     }
 }
 
+// At most 96 registers a thread (which also fits 544 threads, CW = 16, in
+// one CTA): for small buckets two CTAs share an SM
+// (the cut ring), 18 warps, so one of the four schedulers holds 5 of them,
+// and 5 x 96 x 32 registers is what one scheduler's share of the register
+// file (16,384) holds; at 104 the second CTA did not fit and small buckets
+// ran 20-40 % slower at Nd <= 8.
 template <bool OWNER_MAP, int GROUPS, int VW, int SRC = kGradRows, int CW = kConsumerWarps>
-__global__ void __launch_bounds__(32 + 32 * CW, 1)
+__global__ void __maxnreg__(96)
     k_step_tma(const StepArgs a, const Ring ring, const typename ExtraOf<SRC>::type x) {
     constexpr uint32_t kCons = 32u * CW;
     constexpr uint32_t kGroupThreads = kCons / GROUPS;
