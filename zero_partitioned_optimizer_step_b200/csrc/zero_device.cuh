@@ -65,12 +65,6 @@ __device__ __forceinline__ void unpack8(const uint4 x, float f[8]) {
     f[6] = bf16lo(x.w); f[7] = bf16hi(x.w);
 }
 
-__device__ __forceinline__ void add8(float s[8], const uint4 x) {
-    float f[8];
-    unpack8(x, f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) s[e] = __fadd_rn(s[e], f[e]);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // round to nearest even
@@ -124,7 +118,8 @@ __device__ __forceinline__ void adam1(float g_sum, const AdamConsts &c, float &w
 // ---------------------------------------------------------------------------
 // Two fp32 lanes in one 64-bit register, for sm_100's packed fp32 add (one
 // instruction per pair; each lane rounded to nearest exactly as the scalar
-// add).  Used for the rank-order sum only, a chain of adds of loaded values.
+// add).  Used for the rank-order sum only, a chain of adds of loaded values
+// (add8 below, and the bulk-copy kernel's consumers).
 // The multiplications and additions of the Adam update stay scalar
 // (__fmul_rn / __fadd_rn, never contracted): measured on B200 against them,
 // packed multiplies and adds each matched bit for bit alone, but a packed
@@ -148,6 +143,15 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 
 // Two bf16 (one 32-bit word, low half first) as an fp32 pair: exact.
 __device__ __forceinline__ uint64_t f2_bf16x2(uint32_t w) { return f2_pack(bf16lo(w), bf16hi(w)); }
+
+// s[e] += bf16 e of x for 8 consecutive elements, in four packed pairs
+// (each lane rounded as __fadd_rn): one row of the rank-order sum.
+__device__ __forceinline__ void add8(float s[8], const uint4 x) {
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+        f2_unpack(f2_add(f2_pack(s[2 * h], s[2 * h + 1]), f2_bf16x2(w[h])), s[2 * h], s[2 * h + 1]);
+}
 
 // Per-CTA partials of the gradient-norm / overflow reduction, added to slot
 // blockIdx.x (the slots are zeroed at the start of each step).  Fixed order,
