@@ -178,23 +178,8 @@ __device__ __forceinline__ uint4 lds128(const unsigned char *p) {
 // Per-thread vector of VW consecutive elements (VW = 2, 4 or 8): bf16 rows
 // read from shared memory as 4/8/16 bytes, fp32 state as 8/16/32 bytes, and
 // streaming global stores of the same widths.  The host picks VW so that a
-// tile keeps every consumer thread of a group busy.
-template <int VW>
-__device__ __forceinline__ void lds_bf16(const unsigned char *p, float f[VW]) {
-    if constexpr (VW == 2) {
-        const uint32_t x = *reinterpret_cast<const uint32_t *>(p);
-        f[0] = zero_dev::bf16lo(x);
-        f[1] = zero_dev::bf16hi(x);
-    } else if constexpr (VW == 4) {
-        const uint2 x = *reinterpret_cast<const uint2 *>(p);
-        f[0] = zero_dev::bf16lo(x.x); f[1] = zero_dev::bf16hi(x.x);
-        f[2] = zero_dev::bf16lo(x.y); f[3] = zero_dev::bf16hi(x.y);
-    } else {
-        zero_dev::unpack8(*reinterpret_cast<const uint4 *>(p), f);
-    }
-}
-
-// VW bf16 from shared memory as VW / 2 fp32 pairs (exact).
+// tile keeps every consumer thread of a group busy.  The bf16 rows come in
+// as VW / 2 fp32 pairs (exact), for the packed rank-order sum.
 template <int VW>
 __device__ __forceinline__ void lds_bf16x2(const unsigned char *p, uint64_t f[VW / 2]) {
     if constexpr (VW == 2) {
