@@ -92,16 +92,54 @@ PEER_CASES = [
     (54_290, 1, 2, 1 << 20, 64, None),
     (128 * 64 * 3 + 5, 128, 2, 4096, 64, None),
 ]
+GUARD_CASE = (100_003, 7, 3, 999, 1, [10_001, 90_002])
 
 
-@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+def call_means(lp):
+    """Per rank: the mean size of the aligned bodies its zero_step_peers
+    call launches (None for a rank whose parts are all scalar), from the
+    plan's bucket and unit queries."""
+    units = lp.units()
+    out = []
+    for r in range(lp.nd):
+        cols = n = 0
+        for b in range(lp.n_buckets):
+            u = lp.query(Z.ZERO_Q_BUCKET_UNIT, b)
+            lo_b, hi_b = lp.query(Z.ZERO_Q_BUCKET_BEGIN, b), lp.query(Z.ZERO_Q_BUCKET_END, b)
+            _, _, s, U, O = units[u]
+            lo = U + r * s
+            p0, p1 = max(lo_b, lo), min(hi_b, lo + s)
+            vlo, vhi = (p0 + 7) // 8 * 8, p1 // 8 * 8
+            if p0 < p1 and (O - lo) % 8 == 0 and vlo < vhi:
+                cols += vhi - vlo
+                n += 1
+        out.append(cols // n if n else None)
+    return out
+
+
+def use_kernel(monkeypatch, kernel, lp):
+    """tma / ldg: every aligned body in the bulk-copy kernel or in K5.
+    mixed: the library's per-call choice, with its threshold at the middle
+    of the ranks' mean body sizes, so that where those differ some ranks'
+    calls run the bulk-copy kernel and the others K5 in the same step."""
+    if kernel == "mixed":
+        means = sorted({m for m in call_means(lp) if m is not None})
+        monkeypatch.delenv("ZERO_STEP_KERNEL", raising=False)
+        monkeypatch.setenv("ZERO_PEER_RING_MIN", str(means[len(means) // 2] if means else 0))
+    else:
+        monkeypatch.delenv("ZERO_PEER_RING_MIN", raising=False)
+        monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
+
+
+@pytest.mark.parametrize("kernel", ["tma", "ldg", "mixed"])
 @pytest.mark.parametrize("psi,nd,stage,bucket,align,units", PEER_CASES)
 def test_ranks_as_allocations_equal_the_one_gpu_step(psi, nd, stage, bucket, align, units, kernel,
                                                      monkeypatch):
-    """Aligned bodies in the bulk-copy kernel (rows through the peer table)
-    or in K5; both against the one-GPU step."""
-    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
+    """Aligned bodies in the bulk-copy kernel (rows through the peer table),
+    in K5, or each launch in the kernel its size picks; all against the
+    one-GPU step."""
     c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=31)
+    use_kernel(monkeypatch, kernel, c.lp)
     R = Ranks(c)
     for t in (1, 2, 3):
         G = c.grads(t)
@@ -242,12 +280,13 @@ def test_two_processes_share_buffers_through_ipc(case):
     assert all(p.exitcode == 0 for p in procs)
 
 
-@pytest.mark.parametrize("kernel", ["tma", "ldg"])
+@pytest.mark.parametrize("kernel", ["tma", "ldg", "mixed"])
 def test_peer_step_writes_stay_inside_their_buffers(kernel, monkeypatch):
     """Every rank's buffers inside guard zones of a fixed byte pattern."""
     from test_canary_fuzz_gpu import Guarded
-    monkeypatch.setenv("ZERO_STEP_KERNEL", kernel)
-    c = Case(100_003, 7, 3, 999, align=1, units=[10_001, 90_002], config_id=34)
+    psi, nd, stage, bucket, align, units = GUARD_CASE
+    c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=34)
+    use_kernel(monkeypatch, kernel, c.lp)
     R = Ranks(c)
     guarded = []
     for name in ("master", "m", "v", "red", "params", "norm", "ovf", "ws"):

@@ -294,3 +294,20 @@ def test_header_compiles_as_c_and_cpp(tmp_path):
         f.write_text(src.read_text())
         subprocess.run([cc, std, "-Wall", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"), "-c",
                         str(f), "-o", str(tmp_path / (name + ".o"))], check=True)
+
+
+def test_mixed_mode_splits_the_calls():
+    """The GPU parity tests' mixed mode sets the per-call threshold so that
+    some ranks' calls fall on each side of it wherever their mean body
+    sizes differ."""
+    from test_peer_gpu import GUARD_CASE, PEER_CASES, call_means
+
+    split = 0
+    for psi, nd, stage, bucket, align, units in PEER_CASES + [GUARD_CASE]:
+        lp = Z.zero_plan(psi, nd, stage, bucket, align_elems=align, unit_elems=units)
+        means = sorted({m for m in call_means(lp) if m is not None})
+        if len(means) > 1:
+            thr = means[len(means) // 2]
+            assert min(means) < thr <= max(means)
+            split += 1
+    assert split >= 3

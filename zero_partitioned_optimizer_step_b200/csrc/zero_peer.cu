@@ -406,21 +406,41 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
 
     // Aligned bodies: where the parameters are written once (stage 3), in the
     // bulk-copy kernel (rows pulled by 1-D bulk copies through the peer table,
-    // no multicast); with replicas to write, in K5.  Measured with the ranks
-    // as allocations on one GPU, both with programmatic dependent launch: at
-    // stage 3 (1.3B, Nd = 16) 0.945 of copy bandwidth against 0.847 for K5;
-    // with replicas (GPT-2-small, Nd = 8) K5 0.850 against 0.823.  The NVLink
-    // rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg forces
-    // either.  Unaligned edges: K5's scalar twin.
+    // no multicast).  With replicas to write, per call: the bulk-copy kernel
+    // when the call's aligned bodies average at least ring_min columns (32 x
+    // 2048 per SM, the size from which a launch keeps the full ring), else
+    // K5.  One kernel per call: choosing per launch by size, so that a call's
+    // chain mixed the two, ran below both kernels alone.  Measured with the
+    // ranks as allocations on one GPU, both with programmatic dependent
+    // launch, against K5 for every call (fraction of 6650 GB/s copy
+    // bandwidth):
+    //   stage 3 (1.3B, Nd = 16): 0.945 against 0.847;
+    //   Psi = 5e8, Nd = 8, one 62.5M-column launch a call: 0.950 against 0.892;
+    //   Psi = 5e8, Nd = 8, 64 MB buckets: 0.927 against 0.918;
+    //   Psi = 5e8, Nd = 32, 64 MB buckets (18 calls of 32 here): 0.885
+    //   against 0.855;
+    //   Psi = 5e8, Nd = 16, 64 MB buckets: 0.891 against 0.900 (a loss);
+    //   GPT-2-small, Nd = 8, 25M-element buckets (4 calls of 8): 0.825
+    //   against 0.829 (a loss).
+    // The NVLink rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg
+    // forces either for every call; ZERO_PEER_RING_MIN=<columns> moves the
+    // threshold.  Unaligned edges: K5's scalar twin.
     zero_tma::Ring ring{};
     int *err = nullptr;
     st = zero_detail::wait_error_word(&err);
     if (st != ZERO_OK) return st;
     const int choice = zero_ring::kernel_choice();
-    const bool tma = (choice == 2 || (choice == 0 && !replicas)) &&
-                     zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring,
-                                            zero_tma::kConsumerWarps);
+    const bool ring_ok = choice != 1 && zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring,
+                                                               zero_tma::kConsumerWarps);
     ring.bulk_p = 0;  // the peer rows are stored through their pointers
+    uint64_t ring_min = replicas ? 32ull * 2048ull * shapes.sms : 0;
+    if (const char *e = std::getenv("ZERO_PEER_RING_MIN")) {
+        char *end = nullptr;
+        const unsigned long long v = std::strtoull(e, &end, 10);
+        if (end != e) ring_min = v;
+    }
+    if (choice == 2) ring_min = 0;
+    bool use_ring = false;  // set below, once the call's bodies are known
     // Vector launches after the first of the call overlap their predecessor
     // (programmatic dependent launch): consecutive launches of one call share
     // only the norm slots, which every kernel adds to after its predecessor
@@ -434,7 +454,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         x.p0 = p0;
         x.p1 = p1;
         const bool dep = pdl && launches++ > 0;
-        if (vec && tma) {
+        if (vec && use_ring) {
             StepArgs sa{};
             sa.w = x.w;
             sa.m = x.m;
@@ -464,19 +484,42 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         }
         return check_launch("zero_step_peers kernel launch");
     };
-    for (uint64_t bk = first; bk < first + count; ++bk) {
+    // r's part of bucket bk: the logical range [p0, p1) and its 8-aligned
+    // body [vlo, vhi), in the vector kernels when vec_ok
+    struct Part {
+        uint64_t p0, p1, vlo, vhi;
+        int64_t s_shift;
+        bool vec_ok;
+    };
+    auto part_of = [&](uint64_t bk) {
         const zero_detail::BucketRange br = zero_detail::bucket_range(*p, bk);
         const uint32_t u = br.unit;
         const uint64_t s_u = p->unit_shard[u];
         const uint64_t lo = p->unit_base[u] + uint64_t(r) * s_u;  // r's slice of unit u, logical
-        const uint64_t p0 = std::max(br.begin, lo), p1 = std::min(br.end, lo + s_u);
+        Part q{};
+        q.p0 = std::max(br.begin, lo);
+        q.p1 = std::min(br.end, lo + s_u);
+        q.s_shift = int64_t(p->unit_offset[u]) - int64_t(lo);
+        q.vlo = (q.p0 + 7) & ~uint64_t(7);
+        q.vhi = q.p1 & ~uint64_t(7);
+        q.vec_ok = q.p0 < q.p1 && mult8(q.s_shift) && q.vlo < q.vhi;
+        return q;
+    };
+    uint64_t vec_cols = 0, vec_n = 0;
+    for (uint64_t bk = first; bk < first + count; ++bk) {
+        const Part q = part_of(bk);
+        if (q.vec_ok) vec_cols += q.vhi - q.vlo, ++vec_n;
+    }
+    use_ring = ring_ok && vec_n > 0 && vec_cols / vec_n >= ring_min;
+    for (uint64_t bk = first; bk < first + count; ++bk) {
+        const Part q = part_of(bk);
+        const uint64_t p0 = q.p0, p1 = q.p1, vlo = q.vlo, vhi = q.vhi;
         if (p0 >= p1) continue;
-        a.s_shift = int64_t(p->unit_offset[u]) - int64_t(lo);
+        a.s_shift = q.s_shift;
         a.q_shift = replicas ? 0 : a.s_shift;
-        const bool vec_ok = mult8(a.s_shift);
-        const uint64_t vlo = (p0 + 7) & ~uint64_t(7), vhi = p1 & ~uint64_t(7);
+        const bool vec_ok = q.vec_ok;
         const zero_trace::Range rb("bucket %llu", (unsigned long long)bk);
-        if (!vec_ok || vlo >= vhi) {
+        if (!vec_ok) {
             st = launch(p0, p1, false);
         } else {
             st = launch(p0, vlo, false);
