@@ -419,7 +419,7 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
     //   Psi = 5e8, Nd = 8, 64 MB buckets: 0.927 against 0.918;
     //   Psi = 5e8, Nd = 32, 64 MB buckets (18 calls of 32 here): 0.885
     //   against 0.855;
-    //   Psi = 5e8, Nd = 16, 64 MB buckets: 0.891 against 0.900 (a loss);
+    //   Psi = 5e8, Nd = 16, 64 MB buckets: 0.919 against 0.900;
     //   GPT-2-small, Nd = 8, 25M-element buckets (4 calls of 8): 0.825
     //   against 0.829 (a loss).
     // The NVLink rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg
