@@ -882,7 +882,7 @@ def run_peer(args, cfg, rank, world, dist):
         return None
     peak, peak_kind = measured_peak()
     hbm_step = Z.zero_bytes_moved(lp, Z.ZERO_BYTES_HBM_STEP)
-    n_ring, n_k5 = peer_kernel_mix(lp, ranks, cfg["stage"], torch.cuda.get_device_properties(dev).multi_processor_count)
+    n_ring, n_k5 = peer_kernel_mix(lp, ranks)
     kname = ("k_step_tma through the peer table" if n_k5 == 0 else
              "k_step_peer" if n_ring == 0 else
              "k_step_tma through the peer table (%d calls) + k_step_peer (%d calls)" % (n_ring, n_k5))
@@ -920,45 +920,13 @@ def run_peer(args, cfg, rank, world, dist):
     }
 
 
-def peer_kernel_mix(lp, ranks, stage, sms):
+def peer_kernel_mix(lp, ranks):
     """How many of `ranks`' calls of one step run their aligned bodies in
-    the bulk-copy kernel and how many in K5, by zero_step_peers' rule: with
-    replicas to write, a call takes the bulk-copy kernel when its bodies
-    average at least 32 x 2048 columns per SM (ZERO_PEER_RING_MIN moves
-    it), else K5; at stage 3 always the bulk-copy kernel; no bulk-copy ring
-    beyond 64 ranks (32 at stage 3); ZERO_STEP_KERNEL=tma|ldg forces
-    either."""
+    the bulk-copy kernel and how many in K5, as the library reports
+    (zero_step_peers_kernel)."""
     import zero_partitioned_optimizer_step_b200 as Z
-    forced = os.environ.get("ZERO_STEP_KERNEL", "")
-    replicas = stage <= 2
-    ring_ok = forced != "ldg" and lp.nd <= (64 if replicas else 32)
-    ring_min = 32 * 2048 * sms if replicas else 0
-    if os.environ.get("ZERO_PEER_RING_MIN", "").isdigit():
-        ring_min = int(os.environ["ZERO_PEER_RING_MIN"])
-    if forced == "tma":
-        ring_min = 0
-    units = lp.units()
-    n_ring = n_k5 = 0
-    for r in ranks:
-        cols = n = 0
-        for b in range(lp.n_buckets):
-            u = lp.query(Z.ZERO_Q_BUCKET_UNIT, b)
-            lo_b, hi_b = lp.query(Z.ZERO_Q_BUCKET_BEGIN, b), lp.query(Z.ZERO_Q_BUCKET_END, b)
-            _, _, s, U, O = units[u]
-            lo = U + r * s
-            p0, p1 = max(lo_b, lo), min(hi_b, lo + s)
-            vlo, vhi = (p0 + 7) // 8 * 8, p1 // 8 * 8
-            if p0 >= p1 or (O - lo) % 8 or vlo >= vhi:
-                continue
-            cols += vhi - vlo
-            n += 1
-        if n == 0:
-            continue
-        if ring_ok and cols // n >= ring_min:
-            n_ring += 1
-        else:
-            n_k5 += 1
-    return n_ring, n_k5
+    kinds = [Z.zero_step_peers_kernel(lp, r) for r in ranks]
+    return kinds.count("k_step_tma"), kinds.count("k_step_peer")
 
 
 def peer_launches(lp, r):

@@ -81,7 +81,7 @@
 extern "C" {
 #endif
 
-#define ZERO_ABI_VERSION 3
+#define ZERO_ABI_VERSION 4
 
 typedef enum zero_status {
     ZERO_OK = 0,
@@ -407,8 +407,11 @@ typedef struct zero_peer_bufs {
  * 0, Nd > ZERO_MAX_PEERS, rank out of range, a NULL or misaligned entry of
  * grads or params.  ZERO_ECUDA: launch failure.  Aligned bodies run in the
  * bulk-copy kernel, rows pulled by 1-D bulk copies from the peers (never
- * multicast), at stage 3, and in a 16-byte-load kernel when replicas are
- * written; ZERO_STEP_KERNEL=tma|ldg forces either. */
+ * multicast), at stage 3, and with replicas when the call's aligned bodies
+ * average at least 32 x 2048 columns per SM (ZERO_PEER_RING_MIN=<columns>
+ * moves the threshold); other calls run them in a 16-byte-load kernel.
+ * One kernel per call; zero_step_peers_kernel() says which.
+ * ZERO_STEP_KERNEL=tma|ldg forces either. */
 zero_status_t zero_step_peers(const zero_plan_t *plan, const zero_peer_bufs_t *bufs,
                               const zero_adam_t *adam, uint64_t t, uint64_t first_bucket,
                               uint64_t n_buckets, void *stream);
@@ -486,14 +489,26 @@ zero_status_t zero_bytes_moved(const zero_plan_t *plan, zero_bytes_kind_t kind,
  * steps, not inside a captured graph. */
 zero_status_t zero_stream_status(void *stream);
 
+#define ZERO_KERNEL_NONE 0u         /* no aligned body: only the scalar edge kernel runs */
 #define ZERO_KERNEL_BULK_COPY 1u    /* k_step_tma: bulk-copy (TMA) shared-memory ring */
-#define ZERO_KERNEL_VECTOR_LOAD 2u  /* k_step_vec8: 16-byte vector loads */
+#define ZERO_KERNEL_VECTOR_LOAD 2u  /* k_step_vec8 / k_step_peer: 16-byte vector loads */
 
 /* Which kernel zero_step() uses for the aligned bucket bodies of `plan` on
  * the current CUDA device (owner_view as in zero_bufs_t), written to *kind.
  * Queries the device once.  ZERO_EINVAL: NULL argument or owner_view out of
  * range.  ZERO_ECUDA: the device query failed. */
 zero_status_t zero_step_kernel(const zero_plan_t *plan, int32_t owner_view, uint32_t *kind);
+
+/* Which kernel zero_step_peers() uses for the aligned bodies of rank
+ * `rank`'s call over buckets [first_bucket, first_bucket + n_buckets) on the
+ * current CUDA device, written to *kind: ZERO_KERNEL_BULK_COPY,
+ * ZERO_KERNEL_VECTOR_LOAD (k_step_peer), or ZERO_KERNEL_NONE when the call
+ * has no aligned body.  Reads the same environment overrides as the call.
+ * Queries the device once.  ZERO_EINVAL: NULL argument, stage 0,
+ * Nd > ZERO_MAX_PEERS, rank out of range or buckets outside the plan.
+ * ZERO_ECUDA: the device query failed. */
+zero_status_t zero_step_peers_kernel(const zero_plan_t *plan, uint32_t rank, uint64_t first_bucket,
+                                     uint64_t n_buckets, uint32_t *kind);
 
 /* Static text of a status code. */
 const char *zero_status_str(zero_status_t status);

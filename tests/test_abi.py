@@ -28,7 +28,7 @@ def test_library_exports_every_declared_function():
     assert len(names) >= 11
     for n in names:
         assert hasattr(L, n), n
-    assert L.zero_abi_version() == 3
+    assert L.zero_abi_version() == 4
 
 
 def test_status_strings():
@@ -253,7 +253,7 @@ def test_plain_c_caller(tmp_path):
     for u in range(3):
         assert got["st3.unit%d" % u] == "%d %d %d" % (o3.unit_pad[u], o3.unit_shard[u], o3.unit_offset[u])
     assert got["st3.release_unheld"] == "%d ESTATE" % Z.ZERO_ESTATE
-    assert got["abi"] == "3"
+    assert got["abi"] == "4"
 
 
 try:

@@ -140,6 +140,13 @@ def test_ranks_as_allocations_equal_the_one_gpu_step(psi, nd, stage, bucket, ali
     one-GPU step."""
     c = Case(psi, nd, stage, bucket, align=align, units=units, config_id=31)
     use_kernel(monkeypatch, kernel, c.lp)
+    kinds = {Z.zero_step_peers_kernel(c.lp, r) for r in range(nd)} - {None}
+    if kernel == "ldg" or nd > 64:
+        assert kinds <= {"k_step_peer"}
+    elif kernel == "tma":
+        assert kinds <= {"k_step_tma"}
+    elif len({m for m in call_means(c.lp) if m is not None}) > 1:
+        assert kinds == {"k_step_tma", "k_step_peer"}, kinds   # both kernels in one step
     R = Ranks(c)
     for t in (1, 2, 3):
         G = c.grads(t)

@@ -121,6 +121,31 @@ def test_valid_peer_step_without_device_reports_ecuda():
                              None) == Z.ZERO_ECUDA
 
 
+def test_step_peers_kernel_argument_checks():
+    """The kernel query checks its arguments before it looks at the device."""
+    L = Z.lib()
+    out = ctypes.c_uint32()
+    pl = Z.zero_plan(1000, 4, 2, 100)
+    assert L.zero_step_peers_kernel(None, 0, 0, 1, ctypes.byref(out)) == Z.ZERO_EINVAL
+    assert L.zero_step_peers_kernel(pl.handle, 0, 0, 1, None) == Z.ZERO_EINVAL
+    assert L.zero_step_peers_kernel(pl.handle, 4, 0, 1, ctypes.byref(out)) == Z.ZERO_EINVAL
+    assert "rank" in L.zero_last_error().decode()
+    assert L.zero_step_peers_kernel(pl.handle, 0, 1, pl.n_buckets, ctypes.byref(out)) == Z.ZERO_EINVAL
+    assert "bucket" in L.zero_last_error().decode()
+    pl0 = Z.zero_plan(1000, 4, 0, 100)
+    assert L.zero_step_peers_kernel(pl0.handle, 0, 0, 1, ctypes.byref(out)) == Z.ZERO_EINVAL
+    big = Z.zero_plan(129 * 64, 129, 2, 1000)
+    assert L.zero_step_peers_kernel(big.handle, 0, 0, 1, ctypes.byref(out)) == Z.ZERO_EINVAL
+    assert "ZERO_MAX_PEERS" in L.zero_last_error().decode()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="needs a machine without a CUDA device")
+def test_step_peers_kernel_without_device_reports_ecuda():
+    out = ctypes.c_uint32()
+    pl = Z.zero_plan(1000, 4, 2, 100)
+    assert Z.lib().zero_step_peers_kernel(pl.handle, 0, 0, pl.n_buckets, ctypes.byref(out)) == Z.ZERO_ECUDA
+
+
 def test_gather_layer_peers_argument_checks():
     L = Z.lib()
     pl = Z.zero_plan(1000, 4, 3, 100, unit_elems=[400, 600])

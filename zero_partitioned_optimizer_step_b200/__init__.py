@@ -129,6 +129,9 @@ def lib():
         L.zero_bytes_moved.argtypes = [vp, ctypes.c_int, ctypes.c_uint32, ctypes.POINTER(u64)]
         L.zero_step_kernel.restype = st
         L.zero_step_kernel.argtypes = [vp, ctypes.c_int32, ctypes.POINTER(ctypes.c_uint32)]
+        L.zero_step_peers_kernel.restype = st
+        L.zero_step_peers_kernel.argtypes = [vp, ctypes.c_uint32, ctypes.c_uint64, ctypes.c_uint64,
+                                             ctypes.POINTER(ctypes.c_uint32)]
         L.zero_reshard.restype = st
         L.zero_reshard.argtypes = [vp, vp, vp, vp, ctypes.c_uint32, vp]
         L.zero_adam_consts.restype = st
@@ -372,6 +375,7 @@ def zero_gather_layer(plan, unit, owner_params, full_layer, stream=None):
                                    _stream(stream)))
 
 
+ZERO_KERNEL_NONE = 0
 ZERO_KERNEL_BULK_COPY = 1
 ZERO_KERNEL_VECTOR_LOAD = 2
 
@@ -382,6 +386,18 @@ def zero_step_kernel(plan, owner_view=-1):
     out = ctypes.c_uint32()
     _check(lib().zero_step_kernel(plan.handle, int(owner_view), ctypes.byref(out)))
     return "k_step_tma" if out.value == ZERO_KERNEL_BULK_COPY else "k_step_vec8"
+
+
+def zero_step_peers_kernel(plan, rank, first=0, count=None):
+    """Which kernel zero_step_peers runs rank's aligned bodies in, over
+    buckets [first, first + count) (default: the whole step):
+    "k_step_tma" (bulk copies through the peer table), "k_step_peer"
+    (16-byte loads), or None when the call has no aligned body."""
+    if count is None:
+        count = plan.n_buckets - first
+    out = ctypes.c_uint32()
+    _check(lib().zero_step_peers_kernel(plan.handle, int(rank), int(first), int(count), ctypes.byref(out)))
+    return {ZERO_KERNEL_BULK_COPY: "k_step_tma", ZERO_KERNEL_VECTOR_LOAD: "k_step_peer"}.get(out.value)
 
 
 def zero_adam_consts(adam, t, out):

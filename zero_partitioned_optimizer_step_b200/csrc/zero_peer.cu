@@ -350,6 +350,78 @@ zero_status_t validate_peers(const zero_plan_t *p, const zero_peer_bufs_t *b, co
     return ZERO_OK;
 }
 
+// Rank r's part of bucket bk: the logical range [p0, p1) and its 8-aligned
+// body [vlo, vhi), which runs in a vector kernel when vec_ok.
+struct PeerPart {
+    uint64_t p0, p1, vlo, vhi;
+    int64_t s_shift;  // state index = logical index + s_shift
+    bool vec_ok;
+};
+
+PeerPart peer_part(const zero_plan_t &p, uint32_t r, uint64_t bk) {
+    const zero_detail::BucketRange br = zero_detail::bucket_range(p, bk);
+    const uint32_t u = br.unit;
+    const uint64_t s_u = p.unit_shard[u];
+    const uint64_t lo = p.unit_base[u] + uint64_t(r) * s_u;  // r's slice of unit u, logical
+    PeerPart q{};
+    q.p0 = std::max(br.begin, lo);
+    q.p1 = std::min(br.end, lo + s_u);
+    q.s_shift = int64_t(p.unit_offset[u]) - int64_t(lo);
+    q.vlo = (q.p0 + 7) & ~uint64_t(7);
+    q.vhi = q.p1 & ~uint64_t(7);
+    q.vec_ok = q.p0 < q.p1 && mult8(q.s_shift) && q.vlo < q.vhi;
+    return q;
+}
+
+// The kernel of rank r's call over buckets [first, first + count) for its
+// aligned bodies: ZERO_KERNEL_BULK_COPY, ZERO_KERNEL_VECTOR_LOAD (K5), or
+// ZERO_KERNEL_NONE when the call has none.  `ring` receives the bulk-copy
+// ring (err: the device error word its waits report to; may be NULL for a
+// query).
+//
+// Where the parameters are written once (stage 3), the bulk-copy kernel
+// (rows pulled by 1-D bulk copies through the peer table, no multicast).
+// With replicas to write, per call: the bulk-copy kernel when the call's
+// aligned bodies average at least ring_min columns (32 x 2048 per SM, the
+// size from which a launch keeps the full ring), else K5.  One kernel per
+// call: choosing per launch by size, so that a call's chain mixed the two,
+// ran below both kernels alone.  Measured with the ranks as allocations on
+// one GPU, both with programmatic dependent launch, against K5 for every
+// call (fraction of 6650 GB/s copy bandwidth):
+//   stage 3 (1.3B, Nd = 16): 0.945 against 0.847;
+//   Psi = 5e8, Nd = 8, one 62.5M-column launch a call: 0.950 against 0.892;
+//   Psi = 5e8, Nd = 8, 64 MB buckets: 0.927 against 0.918;
+//   Psi = 5e8, Nd = 32, 64 MB buckets (18 calls of 32 here): 0.885
+//   against 0.855;
+//   Psi = 5e8, Nd = 16, 64 MB buckets: 0.919 against 0.900;
+//   GPT-2-small, Nd = 8, 25M-element buckets (4 calls of 8): 0.825
+//   against 0.829 (a loss).
+// The NVLink rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg
+// forces either for every call; ZERO_PEER_RING_MIN=<columns> moves the
+// threshold.  Unaligned edges always run in K5's scalar twin.
+uint32_t peer_call_kernel(const zero_plan_t &p, uint32_t r, uint64_t first, uint64_t count,
+                          const PeerShapes &shapes, int *err, zero_tma::Ring *ring) {
+    const bool replicas = p.stage <= 2;
+    const int choice = zero_ring::kernel_choice();
+    const bool ring_ok = choice != 1 && zero_ring::choose_ring(p.nd, !replicas, shapes.tma_smem, err, ring,
+                                                               zero_tma::kConsumerWarps);
+    ring->bulk_p = 0;  // the peer rows are stored through their pointers
+    uint64_t ring_min = replicas ? 32ull * 2048ull * shapes.sms : 0;
+    if (const char *e = std::getenv("ZERO_PEER_RING_MIN")) {
+        char *end = nullptr;
+        const unsigned long long v = std::strtoull(e, &end, 10);
+        if (end != e) ring_min = v;
+    }
+    if (choice == 2) ring_min = 0;
+    uint64_t vec_cols = 0, vec_n = 0;
+    for (uint64_t bk = first; bk < first + count; ++bk) {
+        const PeerPart q = peer_part(p, r, bk);
+        if (q.vec_ok) vec_cols += q.vhi - q.vlo, ++vec_n;
+    }
+    if (vec_n == 0) return ZERO_KERNEL_NONE;
+    return ring_ok && vec_cols / vec_n >= ring_min ? ZERO_KERNEL_BULK_COPY : ZERO_KERNEL_VECTOR_LOAD;
+}
+
 }  // namespace
 
 ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_bufs_t *b, const zero_adam_t *adam,
@@ -404,43 +476,11 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
             return set_error(ZERO_ECUDA, std::string("zero_step_peers workspace reset: ") + cudaGetErrorString(e));
     }
 
-    // Aligned bodies: where the parameters are written once (stage 3), in the
-    // bulk-copy kernel (rows pulled by 1-D bulk copies through the peer table,
-    // no multicast).  With replicas to write, per call: the bulk-copy kernel
-    // when the call's aligned bodies average at least ring_min columns (32 x
-    // 2048 per SM, the size from which a launch keeps the full ring), else
-    // K5.  One kernel per call: choosing per launch by size, so that a call's
-    // chain mixed the two, ran below both kernels alone.  Measured with the
-    // ranks as allocations on one GPU, both with programmatic dependent
-    // launch, against K5 for every call (fraction of 6650 GB/s copy
-    // bandwidth):
-    //   stage 3 (1.3B, Nd = 16): 0.945 against 0.847;
-    //   Psi = 5e8, Nd = 8, one 62.5M-column launch a call: 0.950 against 0.892;
-    //   Psi = 5e8, Nd = 8, 64 MB buckets: 0.927 against 0.918;
-    //   Psi = 5e8, Nd = 32, 64 MB buckets (18 calls of 32 here): 0.885
-    //   against 0.855;
-    //   Psi = 5e8, Nd = 16, 64 MB buckets: 0.919 against 0.900;
-    //   GPT-2-small, Nd = 8, 25M-element buckets (4 calls of 8): 0.825
-    //   against 0.829 (a loss).
-    // The NVLink rate of either is not measured.  ZERO_STEP_KERNEL=tma|ldg
-    // forces either for every call; ZERO_PEER_RING_MIN=<columns> moves the
-    // threshold.  Unaligned edges: K5's scalar twin.
     zero_tma::Ring ring{};
     int *err = nullptr;
     st = zero_detail::wait_error_word(&err);
     if (st != ZERO_OK) return st;
-    const int choice = zero_ring::kernel_choice();
-    const bool ring_ok = choice != 1 && zero_ring::choose_ring(p->nd, !replicas, shapes.tma_smem, err, &ring,
-                                                               zero_tma::kConsumerWarps);
-    ring.bulk_p = 0;  // the peer rows are stored through their pointers
-    uint64_t ring_min = replicas ? 32ull * 2048ull * shapes.sms : 0;
-    if (const char *e = std::getenv("ZERO_PEER_RING_MIN")) {
-        char *end = nullptr;
-        const unsigned long long v = std::strtoull(e, &end, 10);
-        if (end != e) ring_min = v;
-    }
-    if (choice == 2) ring_min = 0;
-    bool use_ring = false;  // set below, once the call's bodies are known
+    const bool use_ring = peer_call_kernel(*p, r, first, count, shapes, err, &ring) == ZERO_KERNEL_BULK_COPY;
     // Vector launches after the first of the call overlap their predecessor
     // (programmatic dependent launch): consecutive launches of one call share
     // only the norm slots, which every kernel adds to after its predecessor
@@ -484,35 +524,8 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         }
         return check_launch("zero_step_peers kernel launch");
     };
-    // r's part of bucket bk: the logical range [p0, p1) and its 8-aligned
-    // body [vlo, vhi), in the vector kernels when vec_ok
-    struct Part {
-        uint64_t p0, p1, vlo, vhi;
-        int64_t s_shift;
-        bool vec_ok;
-    };
-    auto part_of = [&](uint64_t bk) {
-        const zero_detail::BucketRange br = zero_detail::bucket_range(*p, bk);
-        const uint32_t u = br.unit;
-        const uint64_t s_u = p->unit_shard[u];
-        const uint64_t lo = p->unit_base[u] + uint64_t(r) * s_u;  // r's slice of unit u, logical
-        Part q{};
-        q.p0 = std::max(br.begin, lo);
-        q.p1 = std::min(br.end, lo + s_u);
-        q.s_shift = int64_t(p->unit_offset[u]) - int64_t(lo);
-        q.vlo = (q.p0 + 7) & ~uint64_t(7);
-        q.vhi = q.p1 & ~uint64_t(7);
-        q.vec_ok = q.p0 < q.p1 && mult8(q.s_shift) && q.vlo < q.vhi;
-        return q;
-    };
-    uint64_t vec_cols = 0, vec_n = 0;
     for (uint64_t bk = first; bk < first + count; ++bk) {
-        const Part q = part_of(bk);
-        if (q.vec_ok) vec_cols += q.vhi - q.vlo, ++vec_n;
-    }
-    use_ring = ring_ok && vec_n > 0 && vec_cols / vec_n >= ring_min;
-    for (uint64_t bk = first; bk < first + count; ++bk) {
-        const Part q = part_of(bk);
+        const PeerPart q = peer_part(*p, r, bk);
         const uint64_t p0 = q.p0, p1 = q.p1, vlo = q.vlo, vhi = q.vhi;
         if (p0 >= p1) continue;
         a.s_shift = q.s_shift;
@@ -535,6 +548,23 @@ ZERO_API zero_status_t zero_step_peers(const zero_plan_t *p, const zero_peer_buf
         st = check_launch("zero_step_peers finalize launch");
         if (st != ZERO_OK) return st;
     }
+    return ZERO_OK;
+}
+
+ZERO_API zero_status_t zero_step_peers_kernel(const zero_plan_t *p, uint32_t rank, uint64_t first,
+                                              uint64_t count, uint32_t *kind) {
+    zero_detail::clear_error();
+    if (!p || !kind) return set_error(ZERO_EINVAL, "zero_step_peers_kernel: NULL argument");
+    if (p->stage == 0) return set_error(ZERO_EINVAL, "zero_step_peers_kernel: stage 0 has no owners");
+    if (p->nd > ZERO_MAX_PEERS) return set_error(ZERO_EINVAL, "zero_step_peers_kernel: nd exceeds ZERO_MAX_PEERS");
+    if (rank >= p->nd) return set_error(ZERO_EINVAL, "zero_step_peers_kernel: rank out of range");
+    if (first > p->n_buckets || count > p->n_buckets - first)
+        return set_error(ZERO_EINVAL, "zero_step_peers_kernel: bucket range outside the plan");
+    PeerShapes shapes;
+    const zero_status_t st = peer_shapes(&shapes);
+    if (st != ZERO_OK) return st;
+    zero_tma::Ring ring{};
+    *kind = peer_call_kernel(*p, rank, first, count, shapes, nullptr, &ring);
     return ZERO_OK;
 }
 
